@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl native|reference]
+
+A step is one pass of the whole layer (route -> permute -> gather -> gate/up
+GEMM -> [FP8 h quant] -> down GEMM -> combine) over one batch of every token
+count of the workload, e.g. T = 1, 4, 16, 64 for the decode workload
+(H=4096, I=14336, E=8, top-2, bf16).  Inputs are seeded synthetic tensors;
+the expert weights (2.8 GB for decode) are larger than the 126 MB L2 and
+four input batches rotate between steps.
+
+Metric: layer tokens/s (whole job, all ranks).  N > 1 runs independent
+replicas, one per GPU (the layer is single-GPU; there is no data-path
+collective), timed on the device and reduced as the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import CONFIGS, make_batch, make_weights  # noqa: E402
+
+WORKLOADS = {
+    "decode": dict(cfg="decode", dtype=0),
+    "prefill": dict(cfg="prefill", dtype=0),
+    "fp8": dict(cfg="fp8", dtype=1),
+    "skewed": dict(cfg="skewed", dtype=0),
+}
+NBATCH = 4
+SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
+
+
+def describe(name):
+    c = CONFIGS[name]
+    d = "fp8 e4m3" if WORKLOADS[name]["dtype"] else "bf16"
+    return (f"{name} {d} H={c['H']} I={c['I']} E={c['E']} top-{c['k']} "
+            f"T={','.join(str(t) for t in c['T'])}")
+
+
+def kernels_per_forward(T, k, fp8):
+    """Kernels one moe_forward launches (the cudaMemsetAsync is not a kernel)."""
+    A = T * k
+    if T <= SMALL_T and A <= CHUNK:
+        n = 1                                   # fused route + permute
+    else:
+        n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
+    n += 2 if fp8 else 1                        # [amax] + gather
+    n += 1                                      # gate/up GEMM
+    n += 1 if fp8 else 0                        # h quantisation
+    n += 2                                      # down GEMM + combine
+    return n
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid, self.proc, self.lines = uuid, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def gate_up_bytes(T, k, H, I, active, fp8):
+    """Algorithmic bytes of one gate/up launch: the active experts' W_g and W_u,
+    the T*k gathered activation rows read, the T*k rows of h written (bf16)."""
+    wb = 1 if fp8 else 2
+    return active * 2 * H * I * wb + T * k * H * wb + T * k * I * 2
+
+
+def oracle_sample(W, dtype, Ts, budget_s=12.0):
+    """The oracle on a bounded sample: tokens of the largest batch, one by one,
+    until the time budget is spent.  Returns (tokens/s, cores, description)."""
+    import numpy as np
+    import oracle
+    T = max(Ts)
+    x, logits = make_batch(W, T, 0, 0)
+    ids, w = oracle.route_topk(logits, W.k)
+    used = sorted(set(int(e) for e in np.unique(ids)))
+    remap = {e: i for i, e in enumerate(used)}
+    Wg = W.Wg[used].cpu().to(torch.bfloat16)
+    Wu = W.Wu[used].cpu().to(torch.bfloat16)
+    Wd = W.Wd[used].cpu().to(torch.bfloat16)
+    lid = np.vectorize(remap.get)(ids).astype(np.int32)
+    n, t0 = 0, time.perf_counter()
+    step = max(1, oracle.num_threads())
+    while True:
+        toks = [(n + i) % T for i in range(step)]
+        if dtype == 0:
+            oracle.moe_layer(x, lid, w, Wg, Wu, Wd, tokens=toks)
+        else:   # the FP8 oracle needs every h row for its scale: whole batch
+            oracle.moe_layer_fp8(x, lid, w, Wg, Wu, Wd, tokens=toks)
+            n += T - step
+        n += step
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    what = (f"oracle layer on {n} tokens of the T={T} batch ({budget_s:.0f} s budget), "
+            f"{len(used)} experts")
+    return n / el, oracle.num_threads(), what
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    W = make_weights(wl["cfg"], 0, "cpu")
+    Ts = CONFIGS[wl["cfg"]]["T"]
+    budget = args.ref_step_seconds
+    for _ in range(args.warmup):
+        oracle_sample(W, wl["dtype"], Ts, budget_s=min(1.0, budget))
+    vals, cores, what = [], 1, ""
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, cores, what = oracle_sample(W, wl["dtype"], Ts, budget_s=budget)
+        vals.append(v)
+    el = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    line = {"metric": "fused-MoE layer tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": describe(args.workload)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": what},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args):
+    import mixture_experts_expert_route_b200 as moe
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = WORKLOADS[args.workload]
+    name, dtype = wl["cfg"], wl["dtype"]
+    cfg = CONFIGS[name]
+    Ts = cfg["T"]
+    k, E, H, I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
+    W = make_weights(name, 0, "cuda" if name == "skewed" else "cpu")
+    Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (W.Wg, W.Wu, W.Wd))
+    layer = moe.MoELayer(Wg, Wu, Wd, k=k, dtype=dtype)
+    del Wg, Wu, Wd
+    batches = {T: [make_batch(W, T, 0, b) for b in range(NBATCH)] for T in Ts}
+    dev_in = {T: [(x.to(dev), lg.to(dev)) for x, lg in batches[T]] for T in Ts}
+    outs = {T: torch.empty((T, H), dtype=torch.bfloat16, device=dev) for T in Ts}
+    for T in Ts:
+        layer.workspace(T)
+    stream = torch.cuda.current_stream()
+
+    # active experts of every batch (for the algorithmic bytes)
+    active = {}
+    for T in Ts:
+        active[T] = []
+        for x, lg in dev_in[T]:
+            ids, _ = moe.route_topk(lg, k)
+            active[T].append(int(torch.unique(ids).numel()))
+
+    def step(i, ev=None):
+        for T in Ts:
+            x, lg = dev_in[T][i % NBATCH]
+            layer(x, lg, out=outs[T], events=None if ev is None else ev[T])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if layer.check() != 0:
+        raise RuntimeError("device status word reports a fault")
+
+    evs = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(7)] for T in Ts}
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    uuid = torch.cuda.get_device_properties(dev).uuid
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(f"GPU-{uuid}") as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if layer.check() != 0:
+        raise RuntimeError("device status word reports a fault")
+    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(el, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(el.item())
+    tokens_per_step = sum(Ts)
+    value = tokens_per_step * args.steps * world / (elapsed_ms / 1e3)
+
+    # per-stage device times from the events recorded inside the timed region
+    stage = {T: [[] for _ in range(6)] for T in Ts}
+    for i in range(args.steps):
+        for T in Ts:
+            e = evs[i][T]
+            for s in range(6):
+                stage[T][s].append(e[s].elapsed_time(e[s + 1]))
+    gu_ms = {T: statistics.mean(stage[T][2]) for T in Ts}
+    dn_ms = {T: statistics.mean(stage[T][4]) for T in Ts}
+    layer_ms = {T: statistics.mean([sum(stage[T][s][j] for s in range(6))
+                                    for j in range(args.steps)]) for T in Ts}
+    fp8 = dtype == 1
+    gu_bytes = {T: statistics.mean(gate_up_bytes(T, k, H, I, a, fp8) for a in active[T])
+                for T in Ts}
+    tot_bytes = sum(gu_bytes[T] for T in Ts)
+    tot_ms = sum(gu_ms[T] for T in Ts)
+    hbm, tf, src = peaks()
+    achieved = tot_bytes / (tot_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": None,
+                "kernel": "grouped_gemm_kernel<bf16, gate/up>" if not fp8
+                else "grouped_gemm_kernel<e4m3, gate/up>",
+                "peak_source": src}
+    wb = 1 if fp8 else 2
+    per_T = {}
+    for T in Ts:
+        a = statistics.mean(active[T])
+        layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
+        per_T[str(T)] = {"layer_us": round(1e3 * layer_ms[T], 2),
+                         "gate_up_us": round(1e3 * gu_ms[T], 2),
+                         "down_us": round(1e3 * dn_ms[T], 2),
+                         "active_experts": a,
+                         "layer_hbm_gbs": round(layer_bytes / (layer_ms[T] / 1e3) / 1e9, 1),
+                         "layer_hbm_frac": round(layer_bytes / (layer_ms[T] / 1e3) / 1e9 / hbm,
+                                                 4)}
+
+    # end to end through the public call, host buffers, copies in the timed region
+    e2e = None
+    if not args.no_e2e:
+        hx = {T: [x.pin_memory() for x, _ in batches[T]] for T in Ts}
+        hl = {T: [lg.pin_memory() for _, lg in batches[T]] for T in Ts}
+        ho = {T: torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for T in Ts}
+        dx = {T: torch.empty((T, H), dtype=torch.bfloat16, device=dev) for T in Ts}
+        dl = {T: torch.empty((T, E), dtype=torch.float32, device=dev) for T in Ts}
+
+        def e2e_step(i):
+            for T in Ts:
+                dx[T].copy_(hx[T][i % NBATCH], non_blocking=True)
+                dl[T].copy_(hl[T][i % NBATCH], non_blocking=True)
+                layer(dx[T], dl[T], out=outs[T])
+                ho[T].copy_(outs[T], non_blocking=True)
+
+        for i in range(args.warmup):
+            e2e_step(i)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
+        if dist:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_per_step * args.steps * world / (float(e_ms.item()) / 1e3),
+               "unit": "tokens/s",
+               "h2d_bytes_per_step": sum(T * H * 2 + T * E * 4 for T in Ts),
+               "d2h_bytes_per_step": sum(T * H * 2 for T in Ts)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, what = oracle_sample(W, dtype, Ts)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what}
+
+    launches = args.steps * sum(kernels_per_forward(T, k, fp8) for T in Ts)
+    if rank == 0:
+        line = {"metric": "fused-MoE layer tokens/s", "value": value, "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if fp8 else "bf16",
+                "data": "synthetic (seeded; random-init weights of the workload's shape)",
+                "config": {"workload": describe(args.workload), "global_batch": sum(Ts) * world,
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                           "l2": "inputs larger than L2: expert weights "
+                                 f"{3 * E * H * I * wb / 1e9:.2f} GB, {NBATCH} rotating batches",
+                           "per_T": per_T},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-seconds", type=float, default=5.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

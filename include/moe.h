@@ -1,0 +1,243 @@
+/*
+ * moe.h -- C ABI of a B200-native (sm_100a) fused Mixture-of-Experts layer.
+ *
+ * The layer is the "fused MoE" operation: token routing, data reordering and
+ * the experts' computation as one batched GPU operation instead of a loop over
+ * experts ("Az AWS új MoE-optimalizációkkal gyorsítja a SageMaker AI-t",
+ * § "A fused MoE a számítási folyamat több lépését egyesíti").  For tokens
+ * x [T,H] and fp32 router logits [T,E]:
+ *
+ *   ids, w    = top-k of each logits row, softmax over the selected logits
+ *   permute   = group the T*k assignments by expert, padded to block_m rows
+ *   h         = SiLU(x W_g[e]) * (x W_u[e])          per assignment (SwiGLU)
+ *   y         = w * (h W_d[e])
+ *   out[t]    = sum over the token's k assignments of y
+ *
+ * Conventions for every entry point
+ *   - Pointers named as device buffers are device memory of the current CUDA
+ *     device; the caller allocates and owns every buffer.  The library never
+ *     allocates, frees or synchronises, and enqueues work only on the given
+ *     stream (NULL = the legacy default stream).
+ *   - Argument errors are returned synchronously (MOE_ERR_INVALID_ARG,
+ *     MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE) and nothing is launched.
+ *   - A failed launch returns MOE_ERR_CUDA.
+ *   - Faults found on the device (a bounded wait that ran out, an expert id out
+ *     of range) are written to a device status word (int32, 0 = OK, else a
+ *     moe_status code); the first fault wins.  moe_check_status reads it.
+ *   - Device pointers must be 16-byte aligned; all layouts are row-major.
+ *   - T = 0 is a valid no-op.
+ *   - Limits: 1 <= k <= E <= 256; H and I multiples of 64; block_m a multiple
+ *     of 16 (the token granularity of the tensor-core tiles).
+ *   - No global state: calls on different streams may run concurrently.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle types as cudaStream_t / cudaEvent_t, without the CUDA headers. */
+typedef struct CUstream_st* moe_stream_t;
+typedef struct CUevent_st* moe_event_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* bad pointer, size or alignment */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid request outside the supported limits */
+    MOE_ERR_WORKSPACE = 3,    /* workspace missing or too small */
+    MOE_ERR_CUDA = 4,         /* a CUDA call failed */
+    MOE_ERR_TIMEOUT = 5,      /* a bounded device wait ran out (device status) */
+    MOE_ERR_DEVICE = 6        /* a device-side check failed, e.g. id >= E */
+} moe_status;
+
+typedef enum {
+    MOE_BF16 = 0,      /* bf16 weights and activations, fp32 accumulation */
+    MOE_FP8_E4M3 = 1   /* e4m3 weights (one scale per expert matrix) and
+                          activations (one dynamic scale per tensor), fp32
+                          accumulation, bf16 output */
+} moe_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Version string of the library. */
+MOE_API const char* moe_version(void);
+
+/*
+ * a1. Router top-k.  Router selection of the few experts each token activates
+ * ("Amazon SageMaker AIにおけるMixture-of-Expertsカーネル最適化の深掘り",
+ * § "Mixture-of-Experts (MoE) モデルの原理と推論における課題").
+ *   logits  device f32 [T,E]    router logits
+ *   ids     device i32 [T,k]    out: selected experts, larger logit first;
+ *                               equal logits (and -0/+0) lower index first;
+ *                               NaN ranks below every number
+ *   w       device f32 [T,k]    out: softmax over the selected logits
+ * Errors: T < 0, k < 1, k > E, E > 256, NULL pointers -> MOE_ERR_INVALID_ARG.
+ */
+MOE_API moe_status moe_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                          moe_stream_t stream);
+
+/*
+ * a2. Token permutation ("data reordering", same section of the first page
+ * cited above): a stable, atomic-free counting sort of the A = T*k assignments
+ * (flat index f = t*k + j) by expert.
+ *   ids        device i32 [T,k]          expert of each assignment
+ *   counts     device i32 [E]            out: c_e
+ *   offsets    device i32 [E+1]          out: o_0 = 0,
+ *                                        o_{e+1} = o_e + ceil(c_e/block_m)*block_m
+ *   sorted_ids device i32 [capacity]     out: sorted_ids[o_e + r] = the r-th
+ *                                        smallest f routed to e; every other
+ *                                        slot (pads and the tail) = -1
+ *   inv_perm   device i32 [T*k]          out: slot of assignment f
+ *   tiles      device i32 [capacity/block_m] out: expert owning each block_m
+ *                                        rows, -1 past the last
+ *   num_tiles  device i32 [1]            out: o_E / block_m
+ *   capacity   >= moe_permute_capacity(T, k, E, block_m)
+ *   ws         device scratch of moe_align_permute_workspace_size() bytes
+ * Errors: invalid sizes or NULL -> MOE_ERR_INVALID_ARG; capacity too small or
+ * ws too small -> MOE_ERR_WORKSPACE.  An id outside [0,E) is reported in
+ * the status word given to moe_forward/moe_grouped_ffn, not here (it is
+ * skipped, and the results are then incomplete).
+ */
+MOE_API int moe_permute_capacity(int T, int k, int E, int block_m);
+MOE_API size_t moe_align_permute_workspace_size(int T, int k, int E);
+MOE_API moe_status moe_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
+                             int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                             int32_t* inv_perm, int32_t* tiles, int32_t* num_tiles,
+                             int capacity, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * One-time weight packing (not part of the timed layer).  Converts master
+ * weights W_g, W_u [E,H,I] and W_d [E,I,H] (device bf16) into the K-major
+ * layout the tensor-core GEMMs stream:
+ *   W_gu [E][2I][H]: packed row r of expert e holds, for q = r/32, w = r%32,
+ *        column j = 16q + (w%16) of W_g (w < 16) or of W_u (w >= 16)
+ *   W_dn [E][H][I]:  W_d transposed
+ * in bf16 (MOE_BF16) or e4m3 (MOE_FP8_E4M3).  For FP8 each expert matrix gets
+ * scale s = amax/448 (amax = 0 gives 1), codes = round-to-nearest-even of
+ * w/s saturated to +-448, and scales [E][3] = (s_g, s_u, s_d) is written
+ * (device f32); for bf16 scales may be NULL.
+ * Errors: MOE_ERR_INVALID_ARG for bad sizes/pointers.
+ */
+MOE_API size_t moe_packed_weights_size(moe_dtype dtype, int E, int H, int I);
+MOE_API moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const void* Wg,
+                            const void* Wu, const void* Wd, void* packed, float* scales,
+                            moe_stream_t stream);
+
+/*
+ * a3-a6. Grouped expert FFN over the permuted assignments: the expert GEMMs
+ * A[M,K] x B[K,N] ("Ingénierie de kernels Mixture-of-Experts sur Amazon
+ * SageMaker AI"), computed with the expert-weight rows in the tensor core's
+ * M slot and the tokens in N (the operand swap of "A mátrixok felcserélése
+ * jobban kihasználja a Hopper GPU-kat", re-derived for tcgen05), with the
+ * SiLU*up and routing-weight epilogues fused in:
+ *   X_perm[p] = x[sorted_ids[p] / k]      (zero for pads; FP8: quantised
+ *                                           with s_x = amax(x)/448)
+ *   h[p]      = SiLU(X_perm[p] W_g[e]) * (X_perm[p] W_u[e])   (bf16; FP8:
+ *                                           then quantised with s_h)
+ *   y_perm[p] = w[sorted_ids[p]] * (h[p] W_d[e])   (bf16; 0 for pads)
+ * for every row p of expert e's block.  Inputs come from moe_align_permute.
+ * max_ctas > 0 caps the persistent grid (0 = one CTA per SM).
+ * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE
+ * synchronously; device faults in *status (or, if status is NULL, in the
+ * first int32 of ws).
+ */
+typedef struct {
+    moe_dtype dtype;
+    int T, k, E, H, I;
+    int block_m;                /* padding the permutation used */
+    int capacity;               /* rows of sorted_ids / y_perm */
+    const void* x;              /* device bf16 [T,H], token order */
+    const float* w;             /* device f32 [T*k] routing weights */
+    const int32_t* counts;      /* device i32 [E] */
+    const int32_t* offsets;     /* device i32 [E+1] */
+    const int32_t* sorted_ids;  /* device i32 [capacity] */
+    const void* packed;         /* device, from moe_pack_weights */
+    const float* scales;        /* device f32 [E][3] (FP8), NULL for bf16 */
+    void* y_perm;               /* device bf16 [capacity,H], out */
+    int32_t* status;            /* device i32 status word, may be NULL */
+    int max_ctas;               /* 0 = one CTA per SM */
+} moe_ffn_args;
+
+MOE_API size_t moe_grouped_ffn_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,
+                                      int block_m);
+MOE_API moe_status moe_grouped_ffn(const moe_ffn_args* args, void* ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/*
+ * a7. Weighted top-k combine back to token order (the aggregation of the
+ * experts' outputs, "FP8 esetén a Triton backend bizonyult gyorsabbnak"):
+ *   out[t] = sum_{j=0..k-1} y_perm[inv_perm[t*k+j]]   (fp32, in j order)
+ *   y_perm  device bf16 [*, H], inv_perm device i32 [T*k], out device bf16 [T,H]
+ * Errors: MOE_ERR_INVALID_ARG.
+ */
+MOE_API moe_status moe_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
+                       void* out, moe_stream_t stream);
+
+/*
+ * The whole layer in one call: a1 -> a2 -> a3..a6 -> a7 on one stream, with
+ * every intermediate carved from ws (size from moe_forward_workspace_size).
+ *   x        device bf16 [T,H]; logits device f32 [T,E]
+ *   packed / scales  from moe_pack_weights
+ *   out      device bf16 [T,H]
+ *   ids, w   optional device outputs [T,k] (NULL: kept in ws)
+ *   status   optional device status word (NULL: the first int32 of ws)
+ *   block_m  0 selects 16
+ *   events / n_events  optional: if non-NULL, events[i] is recorded on the
+ *            stream after stage i (0 entry, 1 route+permute, 2 gather/quant,
+ *            3 gate/up GEMM, 4 h quant (FP8), 5 down GEMM, 6 combine); used to
+ *            time the stages.  n_events must be 7 when events is non-NULL.
+ * Errors: as for the stages above.
+ */
+typedef struct {
+    moe_dtype dtype;
+    int T, k, E, H, I;
+    int block_m;
+    const void* x;
+    const float* logits;
+    const void* packed;
+    const float* scales;
+    void* out;
+    int32_t* ids;
+    float* w;
+    int32_t* status;
+    int max_ctas;
+    moe_event_t* events;
+    int n_events;
+} moe_forward_args;
+
+MOE_API size_t moe_forward_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,
+                                  int block_m);
+MOE_API moe_status moe_forward(const moe_forward_args* args, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/*
+ * Reads a device status word: synchronises the stream, then returns
+ * MOE_OK or the code the device recorded (MOE_ERR_TIMEOUT, MOE_ERR_DEVICE).
+ * Errors: MOE_ERR_INVALID_ARG for NULL, MOE_ERR_CUDA if the copy fails.
+ */
+MOE_API moe_status moe_check_status(const int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Failure-detection self-test: launches one CTA that waits on a barrier no
+ * one arrives at, with a limit of timeout_us microseconds (1..1000000); when
+ * it runs out the kernel records MOE_ERR_TIMEOUT in *dev_status and returns.
+ * The same bounded-wait routine guards every wait in the GEMM pipeline.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(int32_t* dev_status, int timeout_us, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

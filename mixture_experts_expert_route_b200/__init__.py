@@ -1,0 +1,15 @@
+"""B200-native (sm_100a) fused Mixture-of-Experts layer.
+
+route top-k -> atomic-free permutation -> tcgen05 grouped SwiGLU GEMMs
+(expert-weight rows in the MMA M slot, tokens in N) -> weighted combine,
+behind the C ABI of include/moe.h.  This package is the thin ctypes binding.
+"""
+from ._lib import (BF16, FP8_E4M3, MoEError, MoELayer, align_permute, check_status, combine,
+                   forward, forward_workspace_size, grouped_ffn, grouped_ffn_workspace_size, lib,
+                   pack_weights, permute_capacity, route_topk, selftest_wait_timeout,
+                   status_string, version, LIB_PATH)
+
+__all__ = ["BF16", "FP8_E4M3", "MoEError", "MoELayer", "align_permute", "check_status", "combine",
+           "forward", "forward_workspace_size", "grouped_ffn", "grouped_ffn_workspace_size", "lib",
+           "pack_weights", "permute_capacity", "route_topk", "selftest_wait_timeout",
+           "status_string", "version", "LIB_PATH"]

@@ -1,0 +1,262 @@
+"""ctypes binding of libmoe_b200.so (the C ABI of include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  There is no
+CPU fallback: if the library is missing, importing this module's functions
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+BF16, FP8_E4M3 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+          3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT",
+          6: "MOE_ERR_DEVICE"}
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int
+SZ = ctypes.c_size_t
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class FfnArgs(ctypes.Structure):
+    _fields_ = [("dtype", I32), ("T", I32), ("k", I32), ("E", I32), ("H", I32), ("I", I32),
+                ("block_m", I32), ("capacity", I32), ("x", P), ("w", P), ("counts", P),
+                ("offsets", P), ("sorted_ids", P), ("packed", P), ("scales", P),
+                ("y_perm", P), ("status", P), ("max_ctas", I32)]
+
+
+class ForwardArgs(ctypes.Structure):
+    _fields_ = [("dtype", I32), ("T", I32), ("k", I32), ("E", I32), ("H", I32), ("I", I32),
+                ("block_m", I32), ("x", P), ("logits", P), ("packed", P), ("scales", P),
+                ("out", P), ("ids", P), ("w", P), ("status", P), ("max_ctas", I32),
+                ("events", P), ("n_events", I32)]
+
+
+_SIGS = {
+    "moe_status_string": ([I32], ctypes.c_char_p),
+    "moe_version": ([], ctypes.c_char_p),
+    "moe_route_topk": ([P, I32, I32, I32, P, P, P], I32),
+    "moe_permute_capacity": ([I32, I32, I32, I32], I32),
+    "moe_align_permute_workspace_size": ([I32, I32, I32], SZ),
+    "moe_align_permute": ([P, I32, I32, I32, I32, P, P, P, P, P, P, I32, P, SZ, P], I32),
+    "moe_packed_weights_size": ([I32, I32, I32, I32], SZ),
+    "moe_pack_weights": ([I32, I32, I32, I32, P, P, P, P, P, P], I32),
+    "moe_grouped_ffn_workspace_size": ([I32, I32, I32, I32, I32, I32, I32], SZ),
+    "moe_grouped_ffn": ([ctypes.POINTER(FfnArgs), P, SZ, P], I32),
+    "moe_combine": ([P, P, I32, I32, I32, P, P], I32),
+    "moe_forward_workspace_size": ([I32, I32, I32, I32, I32, I32, I32], SZ),
+    "moe_forward": ([ctypes.POINTER(ForwardArgs), P, SZ, P], I32),
+    "moe_check_status": ([P, P], I32),
+    "moe_selftest_wait_timeout": ([P, I32, P], I32),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m mixture_experts_expert_route_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise MoEError(code, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def version() -> str:
+    return lib().moe_version().decode()
+
+
+def permute_capacity(T: int, k: int, E: int, block_m: int) -> int:
+    return lib().moe_permute_capacity(T, k, E, block_m)
+
+
+def route_topk(logits: torch.Tensor, k: int, ids=None, w=None, stream=None):
+    T, E = logits.shape
+    dev = logits.device
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev) if ids is None else ids
+    w = torch.empty((T, k), dtype=torch.float32, device=dev) if w is None else w
+    _check(lib().moe_route_topk(_ptr(logits), T, E, k, _ptr(ids), _ptr(w), _stream(stream)),
+           "moe_route_topk")
+    return ids, w
+
+
+def align_permute(ids: torch.Tensor, E: int, block_m: int, capacity: int | None = None,
+                  stream=None):
+    T, k = ids.shape
+    dev = ids.device
+    cap = permute_capacity(T, k, E, block_m) if capacity is None else capacity
+    out = dict(counts=torch.empty(E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               sorted_ids=torch.empty(max(cap, 1), dtype=torch.int32, device=dev),
+               inv_perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+               tiles=torch.empty(max(cap // block_m, 1), dtype=torch.int32, device=dev),
+               num_tiles=torch.empty(1, dtype=torch.int32, device=dev))
+    nws = lib().moe_align_permute_workspace_size(T, k, E)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_align_permute(_ptr(ids), T, k, E, block_m, _ptr(out["counts"]),
+                                   _ptr(out["offsets"]), _ptr(out["sorted_ids"]),
+                                   _ptr(out["inv_perm"]), _ptr(out["tiles"]),
+                                   _ptr(out["num_tiles"]), cap, _ptr(ws), nws, _stream(stream)),
+           "moe_align_permute")
+    out["capacity"] = cap
+    out["block_m"] = block_m
+    return out
+
+
+def pack_weights(dtype: int, Wg: torch.Tensor, Wu: torch.Tensor, Wd: torch.Tensor, stream=None):
+    """Packs bf16 master weights once.  Returns (packed uint8 tensor, scales or None)."""
+    E, H, I = Wg.shape
+    for W in (Wg, Wu, Wd):
+        if W.dtype != torch.bfloat16 or not W.is_contiguous():
+            raise ValueError("master weights must be contiguous bf16")
+    n = lib().moe_packed_weights_size(dtype, E, H, I)
+    packed = torch.empty(n, dtype=torch.uint8, device=Wg.device)
+    scales = torch.empty((E, 3), dtype=torch.float32, device=Wg.device) \
+        if dtype == FP8_E4M3 else None
+    _check(lib().moe_pack_weights(dtype, E, H, I, _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(packed),
+                                  _ptr(scales), _stream(stream)), "moe_pack_weights")
+    return packed, scales
+
+
+def grouped_ffn_workspace_size(dtype, T, k, E, H, I, block_m) -> int:
+    return lib().moe_grouped_ffn_workspace_size(dtype, T, k, E, H, I, block_m)
+
+
+def grouped_ffn(dtype: int, x: torch.Tensor, w: torch.Tensor, perm: dict, packed, scales,
+                E: int, I: int, k: int, y_perm=None, status=None, ws=None, max_ctas: int = 0,
+                stream=None):
+    T, H = x.shape
+    bm, cap = perm["block_m"], perm["capacity"]
+    y_perm = torch.empty((max(cap, 1), H), dtype=torch.bfloat16, device=x.device) \
+        if y_perm is None else y_perm
+    n = grouped_ffn_workspace_size(dtype, T, k, E, H, I, bm)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=x.device) if ws is None else ws
+    a = FfnArgs(dtype, T, k, E, H, I, bm, cap, _ptr(x), _ptr(w), _ptr(perm["counts"]),
+                _ptr(perm["offsets"]), _ptr(perm["sorted_ids"]), _ptr(packed), _ptr(scales),
+                _ptr(y_perm), _ptr(status), max_ctas)
+    _check(lib().moe_grouped_ffn(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn")
+    return y_perm, ws
+
+
+def combine(y_perm, inv_perm, T: int, k: int, H: int, out=None, stream=None):
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device) if out is None else out
+    _check(lib().moe_combine(_ptr(y_perm), _ptr(inv_perm), T, k, H, _ptr(out), _stream(stream)),
+           "moe_combine")
+    return out
+
+
+def forward_workspace_size(dtype, T, k, E, H, I, block_m=0) -> int:
+    return lib().moe_forward_workspace_size(dtype, T, k, E, H, I, block_m)
+
+
+def forward(dtype: int, x, logits, packed, scales, E: int, I: int, k: int, out=None, ids=None,
+            w=None, status=None, ws=None, block_m: int = 0, max_ctas: int = 0, events=None,
+            stream=None):
+    """The whole layer.  ``events`` (7 torch.cuda.Event, optional) are recorded after
+    each stage: entry, route+permute, gather, gate/up, h quant, down, combine."""
+    T, H = x.shape
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    n = forward_workspace_size(dtype, T, k, E, H, I, block_m)
+    if ws is None:
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=x.device)
+    ev_arr = None
+    if events is not None:
+        if len(events) != 7:
+            raise ValueError("events must hold 7 torch.cuda.Event")
+        for e in events:
+            if e.cuda_event == 0:  # create lazily-initialised events
+                e.record()
+        ev_arr = (ctypes.c_void_p * 7)(*[e.cuda_event for e in events])
+    a = ForwardArgs(dtype, T, k, E, H, I, block_m, _ptr(x), _ptr(logits), _ptr(packed),
+                    _ptr(scales), _ptr(out), _ptr(ids), _ptr(w), _ptr(status), max_ctas,
+                    ctypes.cast(ev_arr, ctypes.c_void_p) if ev_arr is not None else None,
+                    7 if ev_arr is not None else 0)
+    _check(lib().moe_forward(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_forward")
+    return out
+
+
+def check_status(status: torch.Tensor, stream=None) -> int:
+    return lib().moe_check_status(_ptr(status), _stream(stream))
+
+
+def selftest_wait_timeout(status: torch.Tensor, timeout_us: int, stream=None) -> None:
+    _check(lib().moe_selftest_wait_timeout(_ptr(status), timeout_us, _stream(stream)),
+           "moe_selftest_wait_timeout")
+
+
+class MoELayer:
+    """A fused MoE layer with packed weights and a reusable workspace.
+
+    >>> layer = MoELayer(Wg, Wu, Wd, k=2, dtype=BF16)   # bf16 [E,H,I], [E,I,H] on cuda
+    >>> out = layer(x, logits)                            # x bf16 [T,H], logits f32 [T,E]
+    """
+
+    def __init__(self, Wg, Wu, Wd, k: int, dtype: int = BF16, block_m: int = 0,
+                 max_ctas: int = 0):
+        self.E, self.H, self.I = Wg.shape
+        self.k, self.dtype, self.block_m, self.max_ctas = k, dtype, block_m, max_ctas
+        self.packed, self.scales = pack_weights(dtype, Wg, Wu, Wd)
+        self.device = Wg.device
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._ws = {}
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if T not in self._ws:
+            n = forward_workspace_size(self.dtype, T, self.k, self.E, self.H, self.I,
+                                       self.block_m)
+            self._ws[T] = torch.empty(max(n, 16), dtype=torch.uint8, device=self.device)
+        return self._ws[T]
+
+    def __call__(self, x, logits, out=None, events=None, stream=None):
+        T = x.shape[0]
+        return forward(self.dtype, x, logits, self.packed, self.scales, self.E, self.I,
+                       self.k, out=out, status=self.status, ws=self.workspace(T),
+                       block_m=self.block_m, max_ctas=self.max_ctas, events=events,
+                       stream=stream)
+
+    def check(self) -> int:
+        return check_status(self.status)

@@ -1,0 +1,323 @@
+// elementwise.cu -- the layer's memory-bound steps: a3 gather (+ FP8
+// quantisation of x), a5 FP8 quantisation of h, a7 combine, the one-time
+// weight packing, and the failure-detection self-test.  All are HBM-bound:
+// 16-byte vector accesses, one warp per row, grids sized from the data.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowsPerBlock = kThreads / 32;
+
+// a3: X_perm[p] = x[sorted_ids[p] / k] for p < offsets[E]; pad rows are zero.
+__global__ void __launch_bounds__(kThreads)
+    gather_bf16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
+                       const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
+                       int capacity, uint4* __restrict__ x_perm) {
+    const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (p >= capacity || p >= offsets[E]) return;
+    const int sid = sorted_ids[p];
+    uint4* dst = x_perm + static_cast<long>(p) * vec_per_row;
+    if (sid < 0) {
+        for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const uint4* src = x + static_cast<long>(sid / k) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ float amax8(uint4 v) {
+    float m = 0.0f;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    return m;
+}
+
+// amax over n bf16 values (n % 8 == 0), folded into *amax_bits with atomicMax.
+__global__ void __launch_bounds__(kThreads)
+    amax_bf16_kernel(const uint4* __restrict__ src, long nvec, uint32_t* amax_bits) {
+    float m = 0.0f;
+    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < nvec;
+         i += static_cast<long>(gridDim.x) * kThreads)
+        m = fmaxf(m, amax8(src[i]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    __shared__ float wm[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, wm[i]);
+        atomic_max_nonneg(amax_bits, m);
+    }
+}
+
+__device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = fp8_quant(bf16_lo(w[i]), s);
+        const uint32_t hi = fp8_quant(bf16_hi(w[i]), s);
+        out[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+    }
+    return make_uint2(out[0], out[1]);
+}
+
+// a3 (FP8): X_perm[p] = e4m3(x[sorted_ids[p] / k] / s_x), s_x = amax(x)/448.
+__global__ void __launch_bounds__(kThreads)
+    gather_fp8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
+                      const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
+                      int capacity, const uint32_t* __restrict__ amax_bits,
+                      uint2* __restrict__ x_perm) {
+    const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (p >= capacity || p >= offsets[E]) return;
+    const int sid = sorted_ids[p];
+    uint2* dst = x_perm + static_cast<long>(p) * vec_per_row;
+    if (sid < 0) {
+        for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint2(0, 0);
+        return;
+    }
+    const float s = fp8_scale_from_amax(*amax_bits);
+    const uint4* src = x + static_cast<long>(sid / k) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = quant8(src[v], s);
+}
+
+// a5: rows p < offsets[E] of a bf16 matrix -> e4m3 with s = amax/448.
+__global__ void __launch_bounds__(kThreads)
+    quant_rows_fp8_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ offsets,
+                          int E, int vec_per_row, int capacity,
+                          const uint32_t* __restrict__ amax_bits, uint2* __restrict__ dst) {
+    const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (p >= capacity || p >= offsets[E]) return;
+    const float s = fp8_scale_from_amax(*amax_bits);
+    const uint4* r = src + static_cast<long>(p) * vec_per_row;
+    uint2* d = dst + static_cast<long>(p) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) d[v] = quant8(r[v], s);
+}
+
+// a7: out[t] = sum_j y_perm[inv_perm[t*k + j]] in fp32, j ascending.
+__global__ void __launch_bounds__(kThreads)
+    combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm, int T,
+                   int k, int vec_per_row, uint4* __restrict__ out) {
+    const long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x;
+    if (i >= static_cast<long>(T) * vec_per_row) return;
+    const long t = i / vec_per_row;
+    const int v = static_cast<int>(i - t * vec_per_row);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+        const int p = inv_perm[t * k + j];
+        const uint4 q = y[static_cast<long>(p) * vec_per_row + v];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            acc[2 * c] += bf16_lo(w[c]);
+            acc[2 * c + 1] += bf16_hi(w[c]);
+        }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * c], acc[2 * c + 1]);
+        o[c] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ---- weight packing (one-time)
+// amax of each expert matrix: blockIdx.y = e*3 + m; folded into amax[e*3+m].
+__global__ void __launch_bounds__(kThreads)
+    matrix_amax_kernel(const uint4* __restrict__ Wg, const uint4* __restrict__ Wu,
+                       const uint4* __restrict__ Wd, long vec_per_matrix, uint32_t* amax) {
+    const int em = blockIdx.y, e = em / 3, m = em % 3;
+    const uint4* src = (m == 0 ? Wg : m == 1 ? Wu : Wd) + static_cast<long>(e) * vec_per_matrix;
+    float mx = 0.0f;
+    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < vec_per_matrix;
+         i += static_cast<long>(gridDim.x) * kThreads)
+        mx = fmaxf(mx, amax8(src[i]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    __shared__ float wm[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < kThreads / 32; ++i) mx = fmaxf(mx, wm[i]);
+        atomic_max_nonneg(&amax[em], mx);
+    }
+}
+
+template <bool FP8>
+__device__ __forceinline__ void put(void* base, long idx, __nv_bfloat16 v, float s) {
+    if constexpr (FP8)
+        static_cast<uint8_t*>(base)[idx] = fp8_quant(__bfloat162float(v), s);
+    else
+        static_cast<__nv_bfloat16*>(base)[idx] = v;
+}
+
+// W_gu[e][r][h], r = 32q + w: column 16q + w%16 of W_g (w < 16) or W_u.
+// Block: 32 packed rows (one q) x 64 h.  grid = (2I/32, H/64, E).
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads)
+    pack_gate_up_kernel(const __nv_bfloat16* __restrict__ Wg, const __nv_bfloat16* __restrict__ Wu,
+                        int H, int I, void* packed, const uint32_t* amax) {
+    __shared__ __nv_bfloat16 tile[64][33];
+    const int q = blockIdx.x, h0 = blockIdx.y * 64, e = blockIdx.z;
+    const long mat = static_cast<long>(e) * H * I;
+    for (int i = threadIdx.x; i < 64 * 32; i += kThreads) {
+        const int hh = i / 32, w = i % 32;
+        const __nv_bfloat16* src = (w < 16) ? Wg : Wu;
+        tile[hh][w] = src[mat + static_cast<long>(h0 + hh) * I + 16 * q + (w & 15)];
+    }
+    __syncthreads();
+    const float sg = FP8 ? fp8_scale_from_amax(amax[e * 3 + 0]) : 1.0f;
+    const float su = FP8 ? fp8_scale_from_amax(amax[e * 3 + 1]) : 1.0f;
+    const long out = static_cast<long>(e) * 2 * I * H;
+    for (int i = threadIdx.x; i < 64 * 32; i += kThreads) {
+        const int w = i / 64, hh = i % 64;
+        put<FP8>(packed, out + static_cast<long>(32 * q + w) * H + h0 + hh, tile[hh][w],
+                 w < 16 ? sg : su);
+    }
+}
+
+// W_dn[e][c][n] = W_d[e][n][c].  Block: 32 x 32.  grid = (H/32, I/32, E).
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads)
+    pack_down_kernel(const __nv_bfloat16* __restrict__ Wd, int H, int I, void* packed,
+                     long packed_offset, const uint32_t* amax) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int c0 = blockIdx.x * 32, n0 = blockIdx.y * 32, e = blockIdx.z;
+    const long mat = static_cast<long>(e) * H * I;
+    for (int i = threadIdx.x; i < 32 * 32; i += kThreads) {
+        const int nn = i / 32, cc = i % 32;
+        tile[nn][cc] = Wd[mat + static_cast<long>(n0 + nn) * H + c0 + cc];
+    }
+    __syncthreads();
+    const float sd = FP8 ? fp8_scale_from_amax(amax[e * 3 + 2]) : 1.0f;
+    for (int i = threadIdx.x; i < 32 * 32; i += kThreads) {
+        const int cc = i / 32, nn = i % 32;
+        put<FP8>(packed, packed_offset + mat + static_cast<long>(c0 + cc) * I + n0 + nn,
+                 tile[nn][cc], sd);
+    }
+}
+
+__global__ void amax_to_scale_kernel(float* scales, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) scales[i] = fp8_scale_from_amax(__float_as_uint(scales[i]));
+}
+
+__global__ void wait_timeout_kernel(int32_t* status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // Nothing ever arrives on bar: the bounded wait must give up.
+        if (!mbar_wait(&bar, 0, nullptr, limit_ns)) report(status, MOE_ERR_TIMEOUT);
+        mbar_arrive(&bar);  // complete the phase so the barrier is left idle
+    }
+}
+
+int blocks_for(long n, int per_block, int cap) {
+    long b = (n + per_block - 1) / per_block;
+    if (b < 1) b = 1;
+    return static_cast<int>(b < cap ? b : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
+                               int E, int k, int H, int capacity, void* x_perm, cudaStream_t s) {
+    if (capacity == 0) return cudaSuccess;
+    gather_bf16_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
+        static_cast<const uint4*>(x), sorted_ids, offsets, E, k, H / 8, capacity,
+        static_cast<uint4*>(x_perm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    amax_bf16_kernel<<<blocks_for(n / 8, kThreads * 4, 1184), kThreads, 0, s>>>(
+        static_cast<const uint4*>(src), n / 8, amax_bits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
+                              int E, int k, int H, int capacity, const uint32_t* amax_bits,
+                              void* x_perm, cudaStream_t s) {
+    if (capacity == 0) return cudaSuccess;
+    gather_fp8_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
+        static_cast<const uint4*>(x), sorted_ids, offsets, E, k, H / 8, capacity, amax_bits,
+        static_cast<uint2*>(x_perm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
+                                  int capacity, const uint32_t* amax_bits, void* h_q,
+                                  cudaStream_t s) {
+    if (capacity == 0) return cudaSuccess;
+    quant_rows_fp8_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
+        static_cast<const uint4*>(h), offsets, E, cols / 8, capacity, amax_bits,
+        static_cast<uint2*>(h_q));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
+                           void* out, cudaStream_t s) {
+    const long n = static_cast<long>(T) * (H / 8);
+    if (n == 0) return cudaSuccess;
+    combine_kernel<<<static_cast<unsigned>((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        static_cast<const uint4*>(y_perm), inv_perm, T, k, H / 8, static_cast<uint4*>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, const void* Wu,
+                                const void* Wd, void* packed, float* scales, uint32_t* amax_tmp,
+                                cudaStream_t s) {
+    const auto* g = static_cast<const __nv_bfloat16*>(Wg);
+    const auto* u = static_cast<const __nv_bfloat16*>(Wu);
+    const auto* d = static_cast<const __nv_bfloat16*>(Wd);
+    const long hi = static_cast<long>(H) * I;
+    const long elt = fp8 ? 1 : 2;
+    if (fp8) {
+        cudaError_t err = cudaMemsetAsync(amax_tmp, 0, sizeof(uint32_t) * 3 * E, s);
+        if (err != cudaSuccess) return err;
+        matrix_amax_kernel<<<dim3(blocks_for(hi / 8, kThreads * 8, 64), 3 * E), kThreads, 0, s>>>(
+            reinterpret_cast<const uint4*>(g), reinterpret_cast<const uint4*>(u),
+            reinterpret_cast<const uint4*>(d), hi / 8, amax_tmp);
+        pack_gate_up_kernel<true><<<dim3(2 * I / 32, H / 64, E), kThreads, 0, s>>>(g, u, H, I,
+                                                                                  packed, amax_tmp);
+        pack_down_kernel<true><<<dim3(H / 32, I / 32, E), kThreads, 0, s>>>(
+            d, H, I, packed, 2 * static_cast<long>(E) * hi, amax_tmp);
+        if (static_cast<void*>(scales) != static_cast<void*>(amax_tmp)) {
+            err = cudaMemcpyAsync(scales, amax_tmp, sizeof(float) * 3 * E, cudaMemcpyDeviceToDevice,
+                                  s);
+            if (err != cudaSuccess) return err;
+        }
+        amax_to_scale_kernel<<<(3 * E + 255) / 256, 256, 0, s>>>(scales, 3 * E);
+    } else {
+        pack_gate_up_kernel<false><<<dim3(2 * I / 32, H / 64, E), kThreads, 0, s>>>(
+            g, u, H, I, packed, nullptr);
+        pack_down_kernel<false><<<dim3(H / 32, I / 32, E), kThreads, 0, s>>>(
+            d, H, I, packed, 2 * static_cast<long>(E) * hi, nullptr);
+    }
+    (void)elt;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_selftest(int32_t* status, int timeout_us, cudaStream_t s) {
+    wait_timeout_kernel<<<1, 32, 0, s>>>(status, static_cast<uint64_t>(timeout_us) * 1000ull);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

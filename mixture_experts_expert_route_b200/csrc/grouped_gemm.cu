@@ -1,0 +1,566 @@
+// grouped_gemm.cu -- a4 (gate/up GEMM + SiLU*up) and a6 (down GEMM + routing
+// weight) as one persistent, warp-specialised tcgen05 kernel.
+//
+// The expert GEMM is A[M,K] x B[K,N] with M = tokens, K = hidden and N = the
+// expert's output size ("Ingénierie de kernels Mixture-of-Experts sur Amazon
+// SageMaker AI").  As in the operand swap of "A mátrixok felcserélése jobban
+// kihasználja a Hopper GPU-kat", this kernel puts the expert-weight rows in the
+// tensor core's M slot (128 rows per tile) and the tokens routed to the expert
+// in N (16..256 in steps of 16), so a token count of 1 still fills the M=128
+// datapath and the weights stream at HBM rate.  The same kernel serves decode
+// (N = 16) and prefill (N up to 256) -- there is one code path.
+//
+// Work decomposition ("dynamic scheduling of variable token groups", "FP8
+// esetén a Triton backend bizonyult gyorsabbnak"): for every expert e with
+// c_e tokens, units = ceil(Mw/128) weight tiles x ceil(c_e/nmax) token tiles,
+// each with KB = ceil(K/BK) k-blocks of 128 bytes.  All units' k-blocks form
+// one linear space that is cut into equal contiguous ranges, one per CTA
+// (stream-K).  Units that straddle a range boundary are finished by whichever
+// contributor arrives last, which sums the fp32 partials in CTA order -- a
+// fixed order, so the result does not depend on timing.
+//
+// Roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer (single
+// thread), warp 2 = TMEM allocator, warps 4-7 = epilogue (TMEM lanes 0-127).
+// smem ring of `stages` (A 16 KB + B nmax*128 B), 128-byte swizzle; two TMEM
+// accumulators of nmax fp32 columns so the epilogue of one unit overlaps the
+// main loop of the next.  Every wait is bounded; on expiry the kernel records
+// MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;            // weight rows per tile (UMMA M)
+constexpr int kRowBytes = 128;      // K bytes per stage row (one swizzle atom)
+constexpr int kATileBytes = kBM * kRowBytes;
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;
+constexpr int kMaxStages = 12;
+constexpr int kMinKbPerCta = 4;
+constexpr int kStagingBytes = 4 * 1024;
+constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
+constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
+
+struct GemmArgs {
+    int E, Mw, K, KB, MT, Mvalid;
+    int nmax, box_rows, stages, tmem_cols;
+    int ldo;
+    void* out;
+    const int32_t* counts;
+    const int32_t* offsets;
+    const float* route_w;
+    const int32_t* sorted_ids;
+    const float* w_scales;
+    const uint32_t* act_amax;
+    uint32_t* out_amax;
+    float* partials;
+    int32_t* counters;
+    int32_t* status;
+};
+
+struct Ctl {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int flag;
+    uint32_t prod_pos;   // k-blocks issued by the producer
+    uint32_t mma_pos;    // k-blocks whose full barrier the MMA thread observed
+    uint32_t mma_issued; // 1 once any MMA was issued
+    int scan_tmp[9];
+    int unit_prefix[kMaxExperts + 1];
+    int ntt[kMaxExperts];
+    int cnt[kMaxExperts];
+    int off[kMaxExperts];
+};
+
+struct Seg {
+    int u, kb0, kb1, e, m, b_row, N;
+};
+
+__device__ __forceinline__ int find_expert(const int* prefix, int E, int u) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ Seg make_seg(const Ctl& c, const GemmArgs& g, long long x,
+                                        long long we) {
+    Seg s;
+    s.u = static_cast<int>(x / g.KB);
+    s.kb0 = static_cast<int>(x - static_cast<long long>(s.u) * g.KB);
+    const long long left = we - x;
+    s.kb1 = (g.KB - s.kb0 <= left) ? g.KB : s.kb0 + static_cast<int>(left);
+    s.e = find_expert(c.unit_prefix, g.E, s.u);
+    const int local = s.u - c.unit_prefix[s.e];
+    const int ntt = c.ntt[s.e];
+    s.m = local / ntt;
+    const int nt = local - s.m * ntt;
+    s.b_row = c.off[s.e] + nt * g.nmax;
+    const int rem = c.cnt[s.e] - nt * g.nmax;
+    const int n = rem < g.nmax ? rem : g.nmax;
+    s.N = (n + 15) & ~15;
+    return s;
+}
+
+// CTA whose range [floor(c*L/G), floor((c+1)*L/G)) holds k-block X.
+__device__ __forceinline__ int owner_cta(long long X, long long L, int G) {
+    return static_cast<int>(((X + 1) * G - 1) / L);
+}
+
+__device__ __forceinline__ void named_bar_epi() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
+    report(status, MOE_ERR_TIMEOUT);
+    *reinterpret_cast<volatile int*>(&c.abort) = 1;
+}
+
+template <bool FP8, int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int c0, float (&v)[16],
+                                               float act_scale, uint8_t* staging, float& amax) {
+    const int wq = (threadIdx.x >> 5) - kEpiWarp0;
+    const int lane = threadIdx.x & 31;
+    constexpr unsigned kFull = 0xffffffffu;
+    if constexpr (EPI == 0) {
+        if constexpr (FP8) {
+            const float sw = g.w_scales[s.e * 3 + (lane < 16 ? 0 : 1)] * act_scale;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= sw;
+        }
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + wq * 1024);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float p = __shfl_xor_sync(kFull, v[i], 16);
+            const float gte = lane < 16 ? v[i] : p;
+            const float up = lane < 16 ? p : v[i];
+            const __nv_bfloat16 h = __float2bfloat16_rn(silu(gte) * up);
+            if (lane < 16) {
+                st[i * 16 + lane] = h;
+                if constexpr (FP8) amax = fmaxf(amax, fabsf(__bfloat162float(h)));
+            }
+        }
+        __syncwarp();
+        const int row = s.b_row + c0 + (lane >> 1);
+        const int col = s.m * 64 + 16 * wq + 8 * (lane & 1);
+        const uint4 val = *reinterpret_cast<const uint4*>(st + (lane >> 1) * 16 + 8 * (lane & 1));
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                  static_cast<long>(row) * g.ldo + col) = val;
+        __syncwarp();
+    } else {
+        if constexpr (FP8) {
+            const float sw = g.w_scales[s.e * 3 + 2] * act_scale;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= sw;
+        }
+        float wt = 0.0f;
+        if (lane < 16) {
+            const int sid = g.sorted_ids[s.b_row + c0 + lane];
+            wt = sid >= 0 ? g.route_w[sid] : 0.0f;
+        }
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + wq * 1024);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float wi = __shfl_sync(kFull, wt, i);
+            st[i * 32 + lane] = __float2bfloat16_rn(v[i] * wi);
+        }
+        __syncwarp();
+        const int hcol0 = s.m * kBM + 32 * wq;
+        if (hcol0 < g.Mvalid) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int piece = lane + 32 * t;
+                const int row = piece >> 2, seg = piece & 3;
+                const uint4 val = *reinterpret_cast<const uint4*>(st + row * 32 + 8 * seg);
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                          static_cast<long>(s.b_row + c0 + row) * g.ldo + hcol0 +
+                                          8 * seg) = val;
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <bool FP8, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    extern __shared__ uint8_t dsmem_raw[];
+    __shared__ Ctl ctl;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smA = base;
+    uint8_t* smB = smA + g.stages * kATileBytes;
+    uint8_t* staging = smB + g.stages * g.nmax * kRowBytes;
+    const int b_stage_bytes = g.nmax * kRowBytes;
+
+    // ---- schedule tables: per-expert counts, offsets, token tiles, unit prefix
+    {
+        const int e = threadIdx.x;
+        int units = 0;
+        if (e < g.E) {
+            const int c = g.counts[e];
+            ctl.cnt[e] = c;
+            ctl.off[e] = g.offsets[e];
+            const int nt = (c + g.nmax - 1) / g.nmax;
+            ctl.ntt[e] = nt;
+            units = nt * g.MT;
+        }
+        int inc = units;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) ctl.scan_tmp[warp] = inc;
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < g.stages; ++i) {
+                mbar_init(&ctl.full[i], 1);
+                mbar_init(&ctl.empty[i], 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&ctl.tfull[i], 1);
+                mbar_init(&ctl.tempty[i], 128);
+            }
+            mbar_init(&ctl.drain, 1);
+            fence_mbar_init();
+            ctl.abort = 0;
+            ctl.prod_pos = 0;
+            ctl.mma_pos = 0;
+            ctl.mma_issued = 0;
+        }
+        if (warp == 0 && lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+        }
+        if (warp == 2) {
+            tmem_alloc(&ctl.tmem_base, g.tmem_cols);
+            tmem_relinquish();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = 0;
+            for (int i = 0; i < kThreads / 32; ++i) {
+                const int t = ctl.scan_tmp[i];
+                ctl.scan_tmp[i] = run;
+                run += t;
+            }
+            ctl.scan_tmp[8] = run;
+        }
+        __syncthreads();
+        if (e < g.E) ctl.unit_prefix[e] = ctl.scan_tmp[warp] + inc - units;
+        if (threadIdx.x == 0) ctl.unit_prefix[g.E] = ctl.scan_tmp[8];
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    const long long L = static_cast<long long>(ctl.unit_prefix[g.E]) * g.KB;
+    long long G = (L + kMinKbPerCta - 1) / kMinKbPerCta;
+    if (G > gridDim.x) G = gridDim.x;
+    if (G < 1) G = 1;
+    const int cta = blockIdx.x;
+    const bool active = L > 0 && cta < G;
+    const long long ws = active ? static_cast<long long>(cta) * L / G : 0;
+    const long long we = active ? static_cast<long long>(cta + 1) * L / G : 0;
+    const uint32_t tmem_base = ctl.tmem_base;
+    const int S = g.stages;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && active) {
+            uint32_t it = 0;
+            const int bk_elems = FP8 ? 128 : 64;
+            for (long long x = ws; x < we;) {
+                const Seg s = make_seg(ctl, g, x, we);
+                const int a_row = s.e * g.Mw + s.m * kBM;
+                const int nload = (s.N + g.box_rows - 1) / g.box_rows;
+                const uint32_t bytes = kATileBytes + nload * g.box_rows * kRowBytes;
+                bool ok = true;
+                for (int kb = s.kb0; kb < s.kb1; ++kb, ++it) {
+                    const int st = it % S;
+                    const uint32_t par = ((it / S) & 1u) ^ 1u;
+                    if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
+                        raise_abort(ctl, g.status);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ctl.full[st], bytes);
+                    tma_load_2d(smA + st * kATileBytes, &tmA, &ctl.full[st], kb * bk_elems, a_row,
+                                kEvictFirst);
+                    for (int j = 0; j < nload; ++j)
+                        tma_load_2d(smB + st * b_stage_bytes + j * g.box_rows * kRowBytes, &tmB,
+                                    &ctl.full[st], kb * bk_elems, s.b_row + j * g.box_rows,
+                                    kEvictLast);
+                }
+                if (!ok) break;
+                x += s.kb1 - s.kb0;
+            }
+            ctl.prod_pos = it;
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0 && active) {
+            uint32_t it = 0, si = 0;
+            bool ok = true;
+            for (long long x = ws; x < we && ok; ++si) {
+                const Seg s = make_seg(ctl, g, x, we);
+                const int acc = si & 1;
+                if (!mbar_wait(&ctl.tempty[acc], ((si >> 1) & 1u) ^ 1u, &ctl.abort)) {
+                    raise_abort(ctl, g.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * g.nmax;
+                const uint32_t idesc = make_idesc<FP8>(kBM, s.N);
+                for (int kb = s.kb0; kb < s.kb1; ++kb, ++it) {
+                    const int st = it % S;
+                    if (!mbar_wait(&ctl.full[st], (it / S) & 1u, &ctl.abort)) {
+                        raise_abort(ctl, g.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(smem_u32(smA + st * kATileBytes));
+                    const uint64_t bd = sw128_desc(smem_u32(smB + st * b_stage_bytes));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc,
+                                  (kb > s.kb0 || kk > 0) ? 1u : 0u);
+                    ctl.mma_issued = 1;
+                    umma_commit(&ctl.empty[st]);
+                }
+                if (!ok) break;
+                umma_commit(&ctl.tfull[acc]);
+                x += s.kb1 - s.kb0;
+            }
+            ctl.mma_pos = it;
+        }
+        __syncwarp();
+    } else if (warp >= kEpiWarp0) {
+        // ------------------------------------------------ epilogue
+        const int wq = warp - kEpiWarp0;
+        const int row = 32 * wq + lane;  // accumulator row = TMEM lane
+        float act_scale = 1.0f;
+        if constexpr (FP8) act_scale = fp8_scale_from_amax(*g.act_amax);
+        float amax = 0.0f;
+        uint32_t si = 0;
+        for (long long x = ws; active && x < we; ++si) {
+            const Seg s = make_seg(ctl, g, x, we);
+            const int acc = si & 1;
+            if (!mbar_wait(&ctl.tfull[acc], (si >> 1) & 1u, &ctl.abort)) {
+                raise_abort(ctl, g.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + acc * g.nmax;
+            if (s.kb0 == 0 && s.kb1 == g.KB) {
+                for (int c0 = 0; c0 < s.N; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+                    epilogue_chunk<FP8, EPI>(g, s, c0, v, act_scale, staging, amax);
+                }
+                tc_fence_before();
+                mbar_arrive(&ctl.tempty[acc]);
+            } else {
+                const long long X0 = static_cast<long long>(s.u) * g.KB;
+                const int cf = owner_cta(X0, L, static_cast<int>(G));
+                const int cl = owner_cta(X0 + g.KB - 1, L, static_cast<int>(G));
+                const long long slot_elems = static_cast<long long>(kBM) * g.nmax;
+                float* mine = g.partials + (2LL * cta + (cta == cf ? 1 : 0)) * slot_elems +
+                              static_cast<long long>(row) * g.nmax;
+                for (int c0 = 0; c0 < s.N; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+                    float4* p4 = reinterpret_cast<float4*>(mine + c0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        p4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+                tc_fence_before();
+                mbar_arrive(&ctl.tempty[acc]);
+                __threadfence();
+                named_bar_epi();
+                if (threadIdx.x == kEpiWarp0 * 32) {
+                    const int old = atomicAdd(&g.counters[cf], 1);
+                    ctl.flag = (old == cl - cf) ? 1 : 0;
+                }
+                named_bar_epi();
+                const int finisher = ctl.flag;
+                named_bar_epi();
+                if (finisher) {
+                    __threadfence();
+                    for (int c0 = 0; c0 < s.N; c0 += 16) {
+                        float v[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                        for (int cc = cf; cc <= cl; ++cc) {
+                            const float* p = g.partials +
+                                             (2LL * cc + (cc == cf ? 1 : 0)) * slot_elems +
+                                             static_cast<long long>(row) * g.nmax + c0;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i);
+                        }
+                        epilogue_chunk<FP8, EPI>(g, s, c0, v, act_scale, staging, amax);
+                    }
+                    if (threadIdx.x == kEpiWarp0 * 32) g.counters[cf] = 0;
+                }
+            }
+            x += s.kb1 - s.kb0;
+        }
+        if constexpr (FP8 && EPI == 0) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            if (lane == 0 && amax > 0.0f) atomic_max_nonneg(g.out_amax, amax);
+        }
+    }
+
+    __syncthreads();
+    if (*reinterpret_cast<volatile int*>(&ctl.abort)) {
+        // Drain: wait (bounded) for this CTA's own MMAs and copies in flight.
+        if (warp == 1 && lane == 0 && ctl.mma_issued) {
+            umma_commit(&ctl.drain);
+            mbar_wait(&ctl.drain, 0, nullptr, kDrainLimitNs);
+        }
+        if (warp == 0 && lane == 0) {
+            for (uint32_t it = ctl.mma_pos; it < ctl.prod_pos; ++it)
+                mbar_wait(&ctl.full[it % S], (it / S) & 1u, nullptr, kDrainLimitNs);
+        }
+        __syncthreads();
+    }
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, g.tmem_cols);
+    }
+}
+
+// ---- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int K, long rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * (fp8 ? 1 : 2)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64),
+                               static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP8, int EPI>
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+                     int smem, cudaStream_t s) {
+    auto kern = grouped_gemm_kernel<FP8, EPI>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, smem, s>>>(a, b, g);
+    return cudaGetLastError();
+}
+
+int pow2_at_least(int v) {
+    int p = 32;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+}  // namespace
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n > kMaxCtas ? kMaxCtas : n;
+}
+
+int gemm_nmax_for(int T) {
+    int n = (T + 15) & ~15;
+    if (n < 16) n = 16;
+    return n > 256 ? 256 : n;
+}
+
+size_t gemm_partials_bytes(int nmax) {
+    return static_cast<size_t>(kMaxCtas) * 2 * kBM * nmax * sizeof(float);
+}
+
+cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
+    GemmArgs g{};
+    g.E = p.E;
+    g.Mw = p.Mw;
+    g.K = p.K;
+    const int bk = p.fp8 ? 128 : 64;
+    g.KB = (p.K + bk - 1) / bk;
+    g.MT = (p.Mw + kBM - 1) / kBM;
+    g.Mvalid = p.Mvalid;
+    g.nmax = p.nmax;
+    g.box_rows = p.nmax < 64 ? p.nmax : 64;
+    const int stage_bytes = kATileBytes + p.nmax * kRowBytes;
+    int stages = (kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024 - kStagingBytes - 1024) /
+                 stage_bytes;
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return cudaErrorInvalidValue;
+    g.stages = stages;
+    g.tmem_cols = pow2_at_least(2 * p.nmax);
+    g.ldo = p.ldo;
+    g.out = p.out;
+    g.counts = p.counts;
+    g.offsets = p.offsets;
+    g.route_w = p.route_w;
+    g.sorted_ids = p.sorted_ids;
+    g.w_scales = p.w_scales;
+    g.act_amax = p.act_amax;
+    g.out_amax = p.out_amax;
+    g.partials = p.partials;
+    g.counters = p.counters;
+    g.status = p.status;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, p.weights, p.fp8, p.K, static_cast<long>(p.E) * p.Mw, kBM) ||
+        !make_map(&tb, p.act, p.fp8, p.K, p.capacity, g.box_rows))
+        return cudaErrorInvalidValue;
+    int grid = device_sm_count();
+    if (p.max_ctas > 0 && p.max_ctas < grid) grid = p.max_ctas;
+    const int smem = 1024 + stages * stage_bytes + kStagingBytes;
+    if (p.fp8) {
+        return p.epi == 0 ? launch_t<true, 0>(ta, tb, g, grid, smem, s)
+                          : launch_t<true, 1>(ta, tb, g, grid, smem, s);
+    }
+    return p.epi == 0 ? launch_t<false, 0>(ta, tb, g, grid, smem, s)
+                      : launch_t<false, 1>(ta, tb, g, grid, smem, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,78 @@
+// kernels.h -- host-side launchers of the layer's kernels (internal; the
+// public surface is include/moe.h).  Every launcher enqueues on `stream`,
+// never synchronises and returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- a1/a2 (route_permute.cu)
+cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                              cudaStream_t s);
+// Single-CTA route + permute for small batches (T <= kSmallT, T*k <= kChunk).
+constexpr int kSmallT = 128;
+constexpr int kChunk = 2048;  // assignments per permutation chunk
+int permute_chunks(long A);
+bool fused_route_permute_ok(int T, int k);
+cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k, int block_m,
+                                       int capacity, int32_t* ids, float* w, int32_t* counts,
+                                       int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
+                                       int32_t* tiles, int32_t* num_tiles, int32_t* status,
+                                       cudaStream_t s);
+cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
+                                 int capacity, int32_t* counts, int32_t* offsets,
+                                 int32_t* sorted_ids, int32_t* inv_perm, int32_t* tiles,
+                                 int32_t* num_tiles, int32_t* chunk_counts, int32_t* status,
+                                 cudaStream_t s);
+
+// ---- a3/a5/a7 and packing (elementwise.cu)
+cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
+                               int E, int k, int H, int capacity, void* x_perm, cudaStream_t s);
+cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s);
+cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
+                              int E, int k, int H, int capacity, const uint32_t* amax_bits,
+                              void* x_perm, cudaStream_t s);
+cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
+                                  int capacity, const uint32_t* amax_bits, void* h_q,
+                                  cudaStream_t s);
+cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
+                           void* out, cudaStream_t s);
+cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, const void* Wu,
+                                const void* Wd, void* packed, float* scales, uint32_t* amax_tmp,
+                                cudaStream_t s);
+cudaError_t launch_wait_timeout_selftest(int32_t* status, int timeout_us, cudaStream_t s);
+
+// ---- a4/a6 (grouped_gemm.cu)
+struct GemmProblem {
+    int fp8;              // 0 bf16, 1 e4m3
+    int epi;              // 0: gate/up -> SiLU*up -> h; 1: down -> * w -> y
+    int E, Mw, K;         // weight rows per expert, reduction length
+    int Mvalid;           // weight rows per expert that are real (masking)
+    int nmax;             // token-tile cap (multiple of 16, <= 256)
+    int capacity;         // rows of the activation operand
+    const void* weights;  // packed [E*Mw, K]
+    const void* act;      // [capacity, K]
+    void* out;            // [capacity, ldo] bf16
+    int ldo;
+    const int32_t* counts;
+    const int32_t* offsets;
+    const float* route_w;        // epi 1
+    const int32_t* sorted_ids;   // epi 1
+    const float* w_scales;       // [E][3] (FP8)
+    const uint32_t* act_amax;    // FP8: amax bits of the activation operand
+    uint32_t* out_amax;          // FP8 epi 0: amax of h (bits)
+    float* partials;             // [max_ctas][2][128*nmax] f32
+    int32_t* counters;           // [max_ctas] zeroed
+    int32_t* status;
+    int max_ctas;
+};
+int gemm_nmax_for(int T);
+size_t gemm_partials_bytes(int nmax);
+cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace moe

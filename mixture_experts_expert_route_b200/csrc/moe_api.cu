@@ -1,0 +1,418 @@
+// moe_api.cu -- the extern "C" boundary declared in include/moe.h: argument
+// validation (nothing is launched on a bad argument), workspace carving, and
+// the order of launches on the caller's stream.  Never allocates, never
+// synchronises (except moe_check_status, whose job is to read the device).
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kCtlInts = 640;  // status, amax_x, amax_h, counters (2 x kMaxCtas)
+constexpr int kCtlStatus = 0, kCtlAmaxX = 1, kCtlAmaxH = 2, kCtlCountersGu = 64,
+              kCtlCountersDn = 64 + kMaxCtas;
+static_assert(kCtlCountersDn + kMaxCtas <= kCtlInts, "control block too small");
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status check_route(int T, int E, int k) {
+    if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status check_layer(moe_dtype dt, int T, int k, int E, int H, int I, int block_m) {
+    moe_status s = check_route(T, E, k);
+    if (s != MOE_OK) return s;
+    if (dt != MOE_BF16 && dt != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+    if (H < 64 || I < 64 || block_m < 16) return MOE_ERR_INVALID_ARG;
+    if (H % 64 != 0 || I % 64 != 0 || block_m % 16 != 0) return MOE_ERR_UNSUPPORTED;
+    if (block_m > 4096) return MOE_ERR_UNSUPPORTED;
+    const long long A = static_cast<long long>(T) * k;
+    const long long cap = A + (A < E ? A : E) * (block_m - 1);
+    // row coordinates of the tensor maps and row indices are 32-bit
+    if (cap > (1LL << 30) || static_cast<long long>(E) * 2 * I > (1LL << 30))
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct Carver {
+    char* base;
+    size_t used = 0;
+    template <class T>
+    T* take(size_t bytes) {
+        T* p = reinterpret_cast<T*>(base ? base + used : nullptr);
+        used += align_up(bytes);
+        return p;
+    }
+};
+
+struct FfnBuffers {
+    int32_t* ctl;
+    void* x_perm;
+    void* h;
+    void* h_q;
+    float* partials;
+};
+
+void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int cap, int H, int I, int nmax) {
+    const size_t elt = dt == MOE_FP8_E4M3 ? 1 : 2;
+    b.x_perm = c.take<void>(static_cast<size_t>(cap) * H * elt);
+    b.h = c.take<void>(static_cast<size_t>(cap) * I * 2);
+    b.h_q = dt == MOE_FP8_E4M3 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
+    b.partials = c.take<float>(gemm_partials_bytes(nmax));
+}
+
+// The control block is carved first, so a missing caller status word means
+// the first int32 of the workspace.
+FfnBuffers carve_ffn(Carver& c, moe_dtype dt, int cap, int H, int I, int nmax) {
+    FfnBuffers b;
+    b.ctl = c.take<int32_t>(sizeof(int32_t) * kCtlInts);
+    carve_ffn_rest(c, b, dt, cap, H, I, nmax);
+    return b;
+}
+
+struct FfnCall {
+    moe_dtype dt;
+    int T, k, E, H, I, cap;
+    const void* x;
+    const float* w;
+    const int32_t* counts;
+    const int32_t* offsets;
+    const int32_t* sorted_ids;
+    const void* packed;
+    const float* scales;
+    void* y_perm;
+    int32_t* status;
+    int max_ctas;
+};
+
+void record(moe_event_t* ev, int i, cudaStream_t s) {
+    if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s);
+}
+
+// a3..a6 on carved buffers.  The control block must already be zeroed.
+moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaStream_t s) {
+    const bool fp8 = f.dt == MOE_FP8_E4M3;
+    const int nmax = gemm_nmax_for(f.T);
+    uint32_t* amax_x = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxX);
+    uint32_t* amax_h = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxH);
+    cudaError_t e;
+    if (fp8) {
+        e = launch_amax_bf16(f.x, static_cast<long>(f.T) * f.H, amax_x, s);
+        if (e == cudaSuccess)
+            e = launch_gather_fp8(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, amax_x,
+                                  b.x_perm, s);
+    } else {
+        e = launch_gather_bf16(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, b.x_perm, s);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    record(ev, 2, s);
+
+    const size_t elt = fp8 ? 1 : 2;
+    GemmProblem gu{};
+    gu.fp8 = fp8;
+    gu.epi = 0;
+    gu.E = f.E;
+    gu.Mw = 2 * f.I;
+    gu.K = f.H;
+    gu.Mvalid = 2 * f.I;
+    gu.nmax = nmax;
+    gu.capacity = f.cap;
+    gu.weights = f.packed;
+    gu.act = b.x_perm;
+    gu.out = b.h;
+    gu.ldo = f.I;
+    gu.counts = f.counts;
+    gu.offsets = f.offsets;
+    gu.w_scales = f.scales;
+    gu.act_amax = amax_x;
+    gu.out_amax = amax_h;
+    gu.partials = b.partials;
+    gu.counters = b.ctl + kCtlCountersGu;
+    gu.status = f.status;
+    gu.max_ctas = f.max_ctas;
+    if (launch_grouped_gemm(gu, s) != cudaSuccess) return MOE_ERR_CUDA;
+    record(ev, 3, s);
+
+    if (fp8 && launch_quant_rows_fp8(b.h, f.offsets, f.E, f.I, f.cap, amax_h, b.h_q, s) !=
+                   cudaSuccess)
+        return MOE_ERR_CUDA;
+    record(ev, 4, s);
+
+    GemmProblem dn = gu;
+    dn.epi = 1;
+    dn.Mw = f.H;
+    dn.K = f.I;
+    dn.Mvalid = f.H;
+    dn.weights = static_cast<const char*>(f.packed) + 2 * static_cast<size_t>(f.E) * f.H * f.I * elt;
+    dn.act = fp8 ? b.h_q : b.h;
+    dn.out = f.y_perm;
+    dn.ldo = f.H;
+    dn.route_w = f.w;
+    dn.sorted_ids = f.sorted_ids;
+    dn.act_amax = amax_h;
+    dn.out_amax = nullptr;
+    dn.counters = b.ctl + kCtlCountersDn;
+    if (launch_grouped_gemm(dn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    record(ev, 5, s);
+    return MOE_OK;
+}
+
+size_t ffn_ws_bytes(moe_dtype dt, int T, int k, int E, int H, int I, int block_m) {
+    Carver c{nullptr};
+    const int cap = moe_permute_capacity(T, k, E, block_m);
+    carve_ffn(c, dt, cap, H, I, gemm_nmax_for(T));
+    return c.used;
+}
+
+struct FwdBuffers {
+    int32_t* ids;
+    float* w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* num_tiles;
+    int32_t* sorted_ids;
+    int32_t* inv_perm;
+    int32_t* tiles;
+    int32_t* chunk_counts;
+    void* y_perm;
+    FfnBuffers ffn;
+};
+
+FwdBuffers carve_fwd(Carver& c, moe_dtype dt, int T, int k, int E, int H, int I, int block_m) {
+    FwdBuffers b;
+    const long A = static_cast<long>(T) * k;
+    const int cap = moe_permute_capacity(T, k, E, block_m);
+    b.ffn.ctl = c.take<int32_t>(sizeof(int32_t) * kCtlInts);
+    b.ids = c.take<int32_t>(sizeof(int32_t) * A);
+    b.w = c.take<float>(sizeof(float) * A);
+    b.counts = c.take<int32_t>(sizeof(int32_t) * E);
+    b.offsets = c.take<int32_t>(sizeof(int32_t) * (E + 1));
+    b.num_tiles = c.take<int32_t>(sizeof(int32_t));
+    b.sorted_ids = c.take<int32_t>(sizeof(int32_t) * (cap > 0 ? cap : 1));
+    b.inv_perm = c.take<int32_t>(sizeof(int32_t) * (A > 0 ? A : 1));
+    b.tiles = c.take<int32_t>(sizeof(int32_t) * (cap / block_m + 1));
+    b.chunk_counts = c.take<int32_t>(sizeof(int32_t) * permute_chunks(A) * E);
+    b.y_perm = c.take<void>(static_cast<size_t>(cap) * H * 2);
+    carve_ffn_rest(c, b.ffn, dt, cap, H, I, gemm_nmax_for(T));
+    return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+        case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+moe_status moe_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                          moe_stream_t stream) {
+    moe_status st = check_route(T, E, k);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!logits || !ids || !w) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_route_topk(logits, T, E, k, ids, w, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute_capacity(int T, int k, int E, int block_m) {
+    if (T < 0 || k < 1 || E < 1 || block_m < 1) return -1;
+    const long long A = static_cast<long long>(T) * k;
+    const long long ne = A < E ? A : E;
+    const long long c = A + ne * (block_m - 1);
+    const long long r = (c + block_m - 1) / block_m * block_m;
+    return r > INT32_MAX ? -1 : static_cast<int>(r);
+}
+
+size_t moe_align_permute_workspace_size(int T, int k, int E) {
+    if (T < 0 || k < 1 || E < 1) return 0;
+    const long A = static_cast<long>(T) * k;
+    const int n = permute_chunks(A);
+    return n <= 1 ? 0 : sizeof(int32_t) * static_cast<size_t>(n) * E;
+}
+
+moe_status moe_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
+                             int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                             int32_t* inv_perm, int32_t* tiles, int32_t* num_tiles, int capacity,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_route(T, E, k);
+    if (st != MOE_OK) return st;
+    if (block_m < 1) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !num_tiles || (T > 0 && (!ids || !inv_perm)))
+        return MOE_ERR_INVALID_ARG;
+    const int need = moe_permute_capacity(T, k, E, block_m);
+    if (need < 0) return MOE_ERR_UNSUPPORTED;
+    if (capacity < need) return MOE_ERR_WORKSPACE;
+    if (capacity > 0 && (!sorted_ids || !tiles)) return MOE_ERR_INVALID_ARG;
+    const size_t wsn = moe_align_permute_workspace_size(T, k, E);
+    if (wsn > 0 && (!ws || ws_bytes < wsn)) return MOE_ERR_WORKSPACE;
+    return from_cuda(launch_align_permute(ids, T, k, E, block_m, capacity, counts, offsets,
+                                          sorted_ids, inv_perm, tiles, num_tiles,
+                                          static_cast<int32_t*>(ws), nullptr,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_packed_weights_size(moe_dtype dtype, int E, int H, int I) {
+    if (E < 1 || H < 1 || I < 1) return 0;
+    const size_t elt = dtype == MOE_FP8_E4M3 ? 1 : 2;
+    return 3 * static_cast<size_t>(E) * H * I * elt;
+}
+
+moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const void* Wg, const void* Wu,
+                            const void* Wd, void* packed, float* scales, moe_stream_t stream) {
+    if (dtype != MOE_BF16 && dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || H < 64 || I < 64) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
+    if (!Wg || !Wu || !Wd || !packed) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(Wg) || !aligned16(Wu) || !aligned16(Wd) || !aligned16(packed))
+        return MOE_ERR_INVALID_ARG;
+    const bool fp8 = dtype == MOE_FP8_E4M3;
+    if (fp8 && (!scales || !aligned16(scales))) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_pack_weights(fp8, E, H, I, Wg, Wu, Wd, packed, scales,
+                                         reinterpret_cast<uint32_t*>(scales),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_grouped_ffn_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,
+                                      int block_m) {
+    if (check_layer(dtype, T, k, E, H, I, block_m) != MOE_OK) return 0;
+    return ffn_ws_bytes(dtype, T, k, E, H, I, block_m);
+}
+
+moe_status moe_grouped_ffn(const moe_ffn_args* a, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!a) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_layer(a->dtype, a->T, a->k, a->E, a->H, a->I, a->block_m);
+    if (st != MOE_OK) return st;
+    if (a->T == 0) return MOE_OK;
+    const int need = moe_permute_capacity(a->T, a->k, a->E, a->block_m);
+    if (a->capacity < need) return MOE_ERR_WORKSPACE;
+    if (!a->x || !a->w || !a->counts || !a->offsets || !a->sorted_ids || !a->packed || !a->y_perm)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a->x) || !aligned16(a->packed) || !aligned16(a->y_perm))
+        return MOE_ERR_INVALID_ARG;
+    if (a->dtype == MOE_FP8_E4M3 && !a->scales) return MOE_ERR_INVALID_ARG;
+    if (a->max_ctas < 0) return MOE_ERR_INVALID_ARG;
+    const size_t need_ws = ffn_ws_bytes(a->dtype, a->T, a->k, a->E, a->H, a->I, a->block_m);
+    if (!ws || ws_bytes < need_ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c{static_cast<char*>(ws)};
+    const FfnBuffers b = carve_ffn(c, a->dtype, a->capacity, a->H, a->I, gemm_nmax_for(a->T));
+    if (cudaMemsetAsync(b.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, a->capacity, a->x, a->w, a->counts,
+              a->offsets, a->sorted_ids, a->packed, a->scales, a->y_perm,
+              a->status ? a->status : b.ctl + kCtlStatus, a->max_ctas};
+    return run_ffn(f, b, nullptr, s);
+}
+
+moe_status moe_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H, void* out,
+                       moe_stream_t stream) {
+    if (T < 0 || k < 1 || H < 8 || H % 8) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !inv_perm || !out || !aligned16(y_perm) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_combine(y_perm, inv_perm, T, k, H, out,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_forward_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,
+                                  int block_m) {
+    if (block_m == 0) block_m = 16;
+    if (check_layer(dtype, T, k, E, H, I, block_m) != MOE_OK) return 0;
+    Carver c{nullptr};
+    carve_fwd(c, dtype, T, k, E, H, I, block_m);
+    return c.used;
+}
+
+moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!a) return MOE_ERR_INVALID_ARG;
+    const int block_m = a->block_m == 0 ? 16 : a->block_m;
+    moe_status st = check_layer(a->dtype, a->T, a->k, a->E, a->H, a->I, block_m);
+    if (st != MOE_OK) return st;
+    if (a->events && a->n_events != 7) return MOE_ERR_INVALID_ARG;
+    if (a->max_ctas < 0) return MOE_ERR_INVALID_ARG;
+    if (a->T == 0) return MOE_OK;
+    if (!a->x || !a->logits || !a->packed || !a->out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a->x) || !aligned16(a->packed) || !aligned16(a->out))
+        return MOE_ERR_INVALID_ARG;
+    if (a->dtype == MOE_FP8_E4M3 && !a->scales) return MOE_ERR_INVALID_ARG;
+    Carver probe{nullptr};
+    carve_fwd(probe, a->dtype, a->T, a->k, a->E, a->H, a->I, block_m);
+    if (!ws || ws_bytes < probe.used || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c{static_cast<char*>(ws)};
+    const FwdBuffers b = carve_fwd(c, a->dtype, a->T, a->k, a->E, a->H, a->I, block_m);
+    int32_t* ids = a->ids ? a->ids : b.ids;
+    float* w = a->w ? a->w : b.w;
+    const int cap = moe_permute_capacity(a->T, a->k, a->E, block_m);
+    int32_t* status = a->status ? a->status : b.ffn.ctl + kCtlStatus;
+    moe_event_t* ev = a->events;
+
+    record(ev, 0, s);
+    if (cudaMemsetAsync(b.ffn.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    cudaError_t e;
+    if (fused_route_permute_ok(a->T, a->k)) {
+        e = launch_route_permute_small(a->logits, a->T, a->E, a->k, block_m, cap, ids, w, b.counts,
+                                       b.offsets, b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,
+                                       status, s);
+    } else {
+        e = launch_route_topk(a->logits, a->T, a->E, a->k, ids, w, s);
+        if (e == cudaSuccess)
+            e = launch_align_permute(ids, a->T, a->k, a->E, block_m, cap, b.counts, b.offsets,
+                                     b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,
+                                     b.chunk_counts, status, s);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    record(ev, 1, s);
+    FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, cap, a->x, w, b.counts, b.offsets,
+              b.sorted_ids, a->packed, a->scales, b.y_perm, status, a->max_ctas};
+    st = run_ffn(f, b.ffn, ev, s);
+    if (st != MOE_OK) return st;
+    if (launch_combine(b.y_perm, b.inv_perm, a->T, a->k, a->H, a->out, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    record(ev, 6, s);
+    return MOE_OK;
+}
+
+moe_status moe_check_status(const int32_t* dev_status, moe_stream_t stream) {
+    if (!dev_status) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (v == 0) return MOE_OK;
+    if (v == MOE_ERR_TIMEOUT || v == MOE_ERR_DEVICE) return static_cast<moe_status>(v);
+    return MOE_ERR_DEVICE;
+}
+
+moe_status moe_selftest_wait_timeout(int32_t* dev_status, int timeout_us, moe_stream_t stream) {
+    if (!dev_status || timeout_us < 1 || timeout_us > 1000000) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_wait_timeout_selftest(dev_status, timeout_us,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

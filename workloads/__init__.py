@@ -13,8 +13,10 @@ Workloads (shapes from the five configurations this library is measured on):
   skewed   T=8192, H=7168, I=2048, E=256, k=8   bf16, Zipf(1.2) expert bias
 
 Recipe (identical for every workload):
-  * one torch.Generator seeded with ``seed`` draws, in this order, x, W_r,
-    the bias ranks (skewed only), W_g, W_u, W_d;
+  * weights: one torch.Generator seeded with ``seed`` draws, in this order,
+    W_r, the bias ranks (skewed only), W_g, W_u, W_d (one expert at a time);
+  * inputs: batch b of T tokens is drawn by its own generator seeded
+    batch_seed(seed, T, b), so any number of batches share one weight set;
   * x ~ N(0, 1); W_r ~ N(0, 1/sqrt(H)) (std); W_g, W_u ~ N(0, 1/sqrt(H));
     W_d ~ N(0, 1/sqrt(I)) -- "N(0, 1/sqrt(fan_in))" read as a standard
     deviation, which keeps activations O(1);
@@ -85,38 +87,44 @@ def zipf_bias(E: int, gen: torch.Generator, s: float = ZIPF_S) -> torch.Tensor:
     return (-s * torch.log(rank)).to(torch.float32)
 
 
-def make_layer(name: str, T: int | None = None, seed: int = 0, device: str = "cpu",
-               E: int | None = None, k: int | None = None, H: int | None = None,
-               I: int | None = None, zero_router: bool = False) -> Layer:
-    """Draws one workload.  Keyword overrides give the small variants tests use.
+def batch_seed(seed: int, T: int, batch: int) -> int:
+    """Seed of input batch ``batch`` with T tokens (independent of the weights' draw)."""
+    return seed * 1_000_003 + 7919 * (batch + 1) + T
 
-    ``device`` is where the expert weights are drawn ("cpu" or "cuda"); x, the
-    router and the logits are always drawn on the CPU.  ``zero_router`` sets
-    W_r = 0 (all logits equal), a special case the oracle is pinned on.
-    """
+
+@dataclass
+class Weights:
+    name: str
+    H: int
+    I: int
+    E: int
+    k: int
+    Wg: torch.Tensor           # [E, H, I]
+    Wu: torch.Tensor           # [E, H, I]
+    Wd: torch.Tensor           # [E, I, H]
+    Wr: torch.Tensor           # [H, E] f32 (CPU)
+    bias: torch.Tensor         # [E] f32 (CPU)
+
+
+def make_weights(name: str, seed: int = 0, device: str = "cpu", E: int | None = None,
+                 k: int | None = None, H: int | None = None, I: int | None = None,
+                 zero_router: bool = False) -> Weights:
+    """Router and expert weights of a workload.  Generator(seed) draws, in order,
+    W_r, the Zipf ranks (skewed only), then W_g, W_u, W_d one expert at a time.
+    On a CUDA ``device`` the expert weights come from a CUDA generator seeded
+    seed + 1 (different values, same distribution)."""
     cfg = dict(CONFIGS[name])
     H = H or cfg["H"]
     I = I or cfg["I"]
     E = E or cfg["E"]
     k = k or cfg["k"]
-    T = cfg["T"][0] if T is None else T
     wdtype = torch.float32 if cfg["master"] == "fp32" else torch.bfloat16
-
     gen = torch.Generator(device="cpu").manual_seed(seed)
-    x = _normal(gen, (T, H), 1.0, "cpu", torch.bfloat16)
     Wr = _normal(gen, (H, E), 1.0 / math.sqrt(H), "cpu", torch.float32)
     if zero_router:
         Wr.zero_()
-    if cfg.get("zipf"):
-        bias = zipf_bias(E, gen)
-    else:
-        bias = torch.zeros(E, dtype=torch.float32)
-    logits = (x.to(torch.float64) @ Wr.to(torch.float64)).to(torch.float32) + bias
-
-    if device == "cpu":
-        wgen = gen
-    else:
-        wgen = torch.Generator(device=device).manual_seed(seed + 1)
+    bias = zipf_bias(E, gen) if cfg.get("zipf") else torch.zeros(E, dtype=torch.float32)
+    wgen = gen if device == "cpu" else torch.Generator(device=device).manual_seed(seed + 1)
     Wg = torch.empty((E, H, I), dtype=wdtype, device=device)
     Wu = torch.empty((E, H, I), dtype=wdtype, device=device)
     Wd = torch.empty((E, I, H), dtype=wdtype, device=device)
@@ -124,7 +132,27 @@ def make_layer(name: str, T: int | None = None, seed: int = 0, device: str = "cp
     for W, std in ((Wg, 1.0 / math.sqrt(H)), (Wu, 1.0 / math.sqrt(H)), (Wd, 1.0 / math.sqrt(I))):
         for e in range(E):
             W[e] = _normal(wgen, W.shape[1:], std, device, wdtype)
-    return Layer(name, T, H, I, E, k, x, logits, Wg, Wu, Wd, Wr, bias,
+    return Weights(name, H, I, E, k, Wg, Wu, Wd, Wr, bias)
+
+
+def make_batch(W: Weights, T: int, seed: int = 0, batch: int = 0):
+    """x ~ N(0,1) bf16 [T, H] and logits = f32(x W_r in f64) + bias [T, E] (CPU)."""
+    gen = torch.Generator(device="cpu").manual_seed(batch_seed(seed, T, batch))
+    x = _normal(gen, (T, W.H), 1.0, "cpu", torch.bfloat16)
+    logits = (x.to(torch.float64) @ W.Wr.to(torch.float64)).to(torch.float32) + W.bias
+    return x, logits
+
+
+def make_layer(name: str, T: int | None = None, seed: int = 0, device: str = "cpu",
+               E: int | None = None, k: int | None = None, H: int | None = None,
+               I: int | None = None, zero_router: bool = False) -> Layer:
+    """One workload: its weights plus input batch 0.  Keyword overrides give the
+    small variants the tests use; ``zero_router`` sets W_r = 0 (all logits
+    equal), a special case the oracle is pinned on."""
+    W = make_weights(name, seed, device, E=E, k=k, H=H, I=I, zero_router=zero_router)
+    T = CONFIGS[name]["T"][0] if T is None else T
+    x, logits = make_batch(W, T, seed, 0)
+    return Layer(name, T, W.H, W.I, W.E, W.k, x, logits, W.Wg, W.Wu, W.Wd, W.Wr, W.bias,
                  meta=dict(seed=seed, weight_device=device))
 
 
