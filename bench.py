@@ -41,6 +41,9 @@ WORKLOADS = {
     "skewed": dict(cfg="skewed", dtype=0),
 }
 NBATCH = 4
+# DRAM bytes (read + write) of one gate/up launch from an ncu capture of the
+# same kernel build, keyed by (workload, T); None until captured.
+TRAFFIC = {}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 
 
@@ -72,22 +75,30 @@ class ClockSampler:
          "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, uuid):
-        self.uuid, self.proc, self.lines = uuid, None, []
+        u = str(uuid)
+        self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+        self.proc, self.lines, self.err = None, [], ""
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             threading.Thread(target=self._read, daemon=True).start()
-        except (OSError, ValueError):
-            self.proc = None
+            threading.Thread(target=self._read_err, daemon=True).start()
+            time.sleep(0.3)   # first sample before the timed region starts
+        except (OSError, ValueError) as e:
+            self.proc, self.err = None, str(e)
         return self
 
     def _read(self):
         for ln in self.proc.stdout:
             self.lines.append(ln.strip())
+
+    def _read_err(self):
+        for ln in self.proc.stderr:
+            self.err += ln
 
     def __exit__(self, *a):
         if self.proc:
@@ -112,8 +123,11 @@ class ClockSampler:
             for n, v in zip(names, f[3:7]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+               "reasons": sorted(reasons), "samples": len(sm)}
+        if not sm:
+            out["error"] = (self.err.strip() or "no samples")[:200]
+        return out
 
 
 def peaks():
@@ -210,7 +224,7 @@ def run_native(args):
     wl = WORKLOADS[args.workload]
     name, dtype = wl["cfg"], wl["dtype"]
     cfg = CONFIGS[name]
-    Ts = cfg["T"]
+    Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else cfg["T"]
     k, E, H, I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
     W = make_weights(name, 0, "cuda" if name == "skewed" else "cpu")
     Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (W.Wg, W.Wu, W.Wd))
@@ -282,14 +296,17 @@ def run_native(args):
     fp8 = dtype == 1
     gu_bytes = {T: statistics.mean(gate_up_bytes(T, k, H, I, a, fp8) for a in active[T])
                 for T in Ts}
-    tot_bytes = sum(gu_bytes[T] for T in Ts)
-    tot_ms = sum(gu_ms[T] for T in Ts)
     hbm, tf, src = peaks()
-    achieved = tot_bytes / (tot_ms / 1e3) / 1e9
+    # dominant kernel: the gate/up GEMM; its largest launch (the largest T)
+    Tr = max(Ts)
+    achieved = gu_bytes[Tr] / (gu_ms[Tr] / 1e3) / 1e9
+    agg = sum(gu_bytes[T] for T in Ts) / (sum(gu_ms[T] for T in Ts) / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": None,
-                "kernel": "grouped_gemm_kernel<bf16, gate/up>" if not fp8
-                else "grouped_gemm_kernel<e4m3, gate/up>",
+                "frac": round(achieved / hbm, 4), "traffic": TRAFFIC.get((args.workload, Tr)),
+                "kernel": ("grouped_gemm_kernel<%s, gate/up> at T=%d" %
+                           ("e4m3" if fp8 else "bf16", Tr)),
+                "bytes_per_launch": int(gu_bytes[Tr]),
+                "all_T_achieved": round(agg, 1), "all_T_frac": round(agg / hbm, 4),
                 "peak_source": src}
     wb = 1 if fp8 else 2
     per_T = {}
@@ -375,6 +392,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
+    ap.add_argument("--Ts", default="", help="comma-separated subset of the token counts")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
