@@ -117,6 +117,26 @@ MOE_API moe_status moe_align_permute(const int32_t* ids, int T, int k, int E, in
                              int capacity, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * The same permutation for callers that cannot allocate device memory or pass
+ * a workspace (for example a plugin of an inference runtime that provides no
+ * workspace, or a thread that must not allocate while it enqueues work).  The
+ * pages have no counterpart of this entry point; it is a deployment aid.
+ * Arguments and outputs are those of moe_align_permute without ws/ws_bytes.
+ * Its scratch is a fixed 256 KB device array inside the library (65536
+ * int32 counters, held on every GPU that loads the library until exit), so
+ * ceil(T*k/2048) * E must not exceed 65536; larger problems return
+ * MOE_ERR_WORKSPACE with nothing launched.  The first call on a device looks
+ * up the array's address for that device; make it before any stream capture.
+ * All calls share the array: each overwrites what it reads, but calls that
+ * overlap on the GPU race.
+ */
+MOE_API moe_status moe_align_permute_noalloc(const int32_t* ids, int T, int k, int E,
+                                             int block_m, int32_t* counts, int32_t* offsets,
+                                             int32_t* sorted_ids, int32_t* inv_perm,
+                                             int32_t* tiles, int32_t* num_tiles, int capacity,
+                                             moe_stream_t stream);
+
+/*
  * One-time weight packing (not part of the timed layer).  Converts master
  * weights W_g, W_u [E,H,I] and W_d [E,I,H] (device bf16) into the K-major
  * layout the tensor-core GEMMs stream:

@@ -52,6 +52,7 @@ _SIGS = {
     "moe_permute_capacity": ([I32, I32, I32, I32], I32),
     "moe_align_permute_workspace_size": ([I32, I32, I32], SZ),
     "moe_align_permute": ([P, I32, I32, I32, I32, P, P, P, P, P, P, I32, P, SZ, P], I32),
+    "moe_align_permute_noalloc": ([P, I32, I32, I32, I32, P, P, P, P, P, P, I32, P], I32),
     "moe_packed_weights_size": ([I32, I32, I32, I32], SZ),
     "moe_pack_weights": ([I32, I32, I32, I32, P, P, P, P, P, P], I32),
     "moe_grouped_ffn_workspace_size": ([I32, I32, I32, I32, I32, I32, I32], SZ),
@@ -140,6 +141,28 @@ def align_permute(ids: torch.Tensor, E: int, block_m: int, capacity: int | None 
                                    _ptr(out["inv_perm"]), _ptr(out["tiles"]),
                                    _ptr(out["num_tiles"]), cap, _ptr(ws), nws, _stream(stream)),
            "moe_align_permute")
+    out["capacity"] = cap
+    out["block_m"] = block_m
+    return out
+
+
+def align_permute_noalloc(ids: torch.Tensor, E: int, block_m: int, capacity: int | None = None,
+                          stream=None):
+    """align_permute without a workspace (the library's built-in scratch)."""
+    T, k = ids.shape
+    dev = ids.device
+    cap = permute_capacity(T, k, E, block_m) if capacity is None else capacity
+    out = dict(counts=torch.empty(E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               sorted_ids=torch.empty(max(cap, 1), dtype=torch.int32, device=dev),
+               inv_perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+               tiles=torch.empty(max(cap // block_m, 1), dtype=torch.int32, device=dev),
+               num_tiles=torch.empty(1, dtype=torch.int32, device=dev))
+    _check(lib().moe_align_permute_noalloc(_ptr(ids), T, k, E, block_m, _ptr(out["counts"]),
+                                           _ptr(out["offsets"]), _ptr(out["sorted_ids"]),
+                                           _ptr(out["inv_perm"]), _ptr(out["tiles"]),
+                                           _ptr(out["num_tiles"]), cap, _stream(stream)),
+           "moe_align_permute_noalloc")
     out["capacity"] = cap
     out["block_m"] = block_m
     return out

@@ -12,7 +12,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["route_permute.cu", "elementwise.cu", "grouped_gemm.cu", "moe_api.cu"]
+SOURCES = ["route_permute.cu", "elementwise.cu", "grouped_gemm.cu", "moe_api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 LIB = os.path.join(HERE, "libmoe_b200.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
