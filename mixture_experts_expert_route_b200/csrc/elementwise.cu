@@ -17,6 +17,8 @@ __global__ void __launch_bounds__(kThreads)
     gather_bf16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
                        const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
                        int capacity, uint4* __restrict__ x_perm) {
+    pdl_wait();
+    pdl_trigger();
     const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (p >= capacity || p >= offsets[E]) return;
@@ -44,6 +46,8 @@ __device__ __forceinline__ float amax8(uint4 v) {
 // amax over n bf16 values (n % 8 == 0), folded into *amax_bits with atomicMax.
 __global__ void __launch_bounds__(kThreads)
     amax_bf16_kernel(const uint4* __restrict__ src, long nvec, uint32_t* amax_bits) {
+    pdl_wait();
+    pdl_trigger();
     float m = 0.0f;
     for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < nvec;
          i += static_cast<long>(gridDim.x) * kThreads)
@@ -77,6 +81,8 @@ __global__ void __launch_bounds__(kThreads)
                       const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
                       int capacity, const uint32_t* __restrict__ amax_bits,
                       uint2* __restrict__ x_perm) {
+    pdl_wait();
+    pdl_trigger();
     const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (p >= capacity || p >= offsets[E]) return;
@@ -96,6 +102,8 @@ __global__ void __launch_bounds__(kThreads)
     quant_rows_fp8_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ offsets,
                           int E, int vec_per_row, int capacity,
                           const uint32_t* __restrict__ amax_bits, uint2* __restrict__ dst) {
+    pdl_wait();
+    pdl_trigger();
     const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (p >= capacity || p >= offsets[E]) return;
@@ -109,6 +117,8 @@ __global__ void __launch_bounds__(kThreads)
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm, int T,
                    int k, int vec_per_row, uint4* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     const long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x;
     if (i >= static_cast<long>(T) * vec_per_row) return;
     const long t = i / vec_per_row;
@@ -155,58 +165,55 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <bool FP8>
-__device__ __forceinline__ void put(void* base, long idx, __nv_bfloat16 v, float s) {
-    if constexpr (FP8)
-        static_cast<uint8_t*>(base)[idx] = fp8_quant(__bfloat162float(v), s);
-    else
-        static_cast<__nv_bfloat16*>(base)[idx] = v;
-}
-
-// W_gu[e][r][h], r = 32q + w: column 16q + w%16 of W_g (w < 16) or W_u.
-// Block: 32 packed rows (one q) x 64 h.  grid = (2I/32, H/64, E).
-template <bool FP8>
+// One 16 KB tile of packed weights per CTA: the swizzled shared-memory image
+// of 128 weight rows x 128 bytes of K (see PackedGeom).  GU selects the gate/up
+// matrix, whose packed row R holds column j = 16*(R/32) + R%16 of W_g
+// (R%32 < 16) or W_u; otherwise the down matrix, whose row R is column R of
+// W_d (W_d transposed).  Out-of-range rows and K are zero.
+// grid = (KB, MT, E).
+template <bool FP8, bool GU>
 __global__ void __launch_bounds__(kThreads)
-    pack_gate_up_kernel(const __nv_bfloat16* __restrict__ Wg, const __nv_bfloat16* __restrict__ Wu,
-                        int H, int I, void* packed, const uint32_t* amax) {
-    __shared__ __nv_bfloat16 tile[64][33];
-    const int q = blockIdx.x, h0 = blockIdx.y * 64, e = blockIdx.z;
+    pack_tiles_kernel(const __nv_bfloat16* __restrict__ Wa, const __nv_bfloat16* __restrict__ Wb,
+                      int H, int I, int MT, int KB, uint8_t* __restrict__ out,
+                      const uint32_t* __restrict__ amax) {
+    __shared__ __align__(16) uint8_t tile[kTileBytes];
+    constexpr int BK = FP8 ? 128 : 64;
+    constexpr int EB = FP8 ? 1 : 2;
+    const int kb = blockIdx.x, m = blockIdx.y, e = blockIdx.z;
     const long mat = static_cast<long>(e) * H * I;
-    for (int i = threadIdx.x; i < 64 * 32; i += kThreads) {
-        const int hh = i / 32, w = i % 32;
-        const __nv_bfloat16* src = (w < 16) ? Wg : Wu;
-        tile[hh][w] = src[mat + static_cast<long>(h0 + hh) * I + 16 * q + (w & 15)];
+    float sa = 1.0f, sb = 1.0f;
+    if constexpr (FP8) {
+        sa = fp8_scale_from_amax(amax[e * 3 + (GU ? 0 : 2)]);
+        sb = fp8_scale_from_amax(amax[e * 3 + 1]);
+    }
+    for (int idx = threadIdx.x; idx < kTileRows * BK; idx += kThreads) {
+        const int r = idx % kTileRows, kk = idx / kTileRows;
+        const int R = m * kTileRows + r;
+        const int kg = kb * BK + kk;
+        float v = 0.0f;
+        float sc = sa;
+        if (GU) {
+            const int j = 16 * (R / 32) + (R & 15);
+            const bool up = (R & 31) >= 16;
+            if (R < 2 * I && kg < H) {
+                v = __bfloat162float((up ? Wb : Wa)[mat + static_cast<long>(kg) * I + j]);
+                sc = up ? sb : sa;
+            }
+        } else if (R < H && kg < I) {
+            v = __bfloat162float(Wa[mat + static_cast<long>(kg) * H + R]);
+        }
+        const int o = r * kTileRowBytes + kk * EB;
+        const int sw = o ^ (((o >> 7) & 7) << 4);
+        if constexpr (FP8)
+            tile[sw] = fp8_quant(v, sc);
+        else
+            *reinterpret_cast<__nv_bfloat16*>(tile + sw) = __float2bfloat16_rn(v);
     }
     __syncthreads();
-    const float sg = FP8 ? fp8_scale_from_amax(amax[e * 3 + 0]) : 1.0f;
-    const float su = FP8 ? fp8_scale_from_amax(amax[e * 3 + 1]) : 1.0f;
-    const long out = static_cast<long>(e) * 2 * I * H;
-    for (int i = threadIdx.x; i < 64 * 32; i += kThreads) {
-        const int w = i / 64, hh = i % 64;
-        put<FP8>(packed, out + static_cast<long>(32 * q + w) * H + h0 + hh, tile[hh][w],
-                 w < 16 ? sg : su);
-    }
-}
-
-// W_dn[e][c][n] = W_d[e][n][c].  Block: 32 x 32.  grid = (H/32, I/32, E).
-template <bool FP8>
-__global__ void __launch_bounds__(kThreads)
-    pack_down_kernel(const __nv_bfloat16* __restrict__ Wd, int H, int I, void* packed,
-                     long packed_offset, const uint32_t* amax) {
-    __shared__ __nv_bfloat16 tile[32][33];
-    const int c0 = blockIdx.x * 32, n0 = blockIdx.y * 32, e = blockIdx.z;
-    const long mat = static_cast<long>(e) * H * I;
-    for (int i = threadIdx.x; i < 32 * 32; i += kThreads) {
-        const int nn = i / 32, cc = i % 32;
-        tile[nn][cc] = Wd[mat + static_cast<long>(n0 + nn) * H + c0 + cc];
-    }
-    __syncthreads();
-    const float sd = FP8 ? fp8_scale_from_amax(amax[e * 3 + 2]) : 1.0f;
-    for (int i = threadIdx.x; i < 32 * 32; i += kThreads) {
-        const int cc = i / 32, nn = i % 32;
-        put<FP8>(packed, packed_offset + mat + static_cast<long>(c0 + cc) * I + n0 + nn,
-                 tile[nn][cc], sd);
-    }
+    uint4* dst = reinterpret_cast<uint4*>(
+        out + (static_cast<size_t>(e * MT + m) * KB + kb) * kTileBytes);
+    const uint4* src = reinterpret_cast<const uint4*>(tile);
+    for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads) dst[i] = src[i];
 }
 
 __global__ void amax_to_scale_kernel(float* scales, int n) {
@@ -239,46 +246,42 @@ int blocks_for(long n, int per_block, int cap) {
 cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
                                int E, int k, int H, int capacity, void* x_perm, cudaStream_t s) {
     if (capacity == 0) return cudaSuccess;
-    gather_bf16_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
-        static_cast<const uint4*>(x), sorted_ids, offsets, E, k, H / 8, capacity,
-        static_cast<uint4*>(x_perm));
-    return cudaGetLastError();
+    return launch_pdl(gather_bf16_kernel, dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock),
+                      dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
+                      k, H / 8, capacity, static_cast<uint4*>(x_perm));
 }
 
 cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s) {
     if (n == 0) return cudaSuccess;
-    amax_bf16_kernel<<<blocks_for(n / 8, kThreads * 4, 1184), kThreads, 0, s>>>(
-        static_cast<const uint4*>(src), n / 8, amax_bits);
-    return cudaGetLastError();
+    return launch_pdl(amax_bf16_kernel, dim3(blocks_for(n / 8, kThreads * 4, 1184)),
+                      dim3(kThreads), 0, s, static_cast<const uint4*>(src), n / 8, amax_bits);
 }
 
 cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
                               int E, int k, int H, int capacity, const uint32_t* amax_bits,
                               void* x_perm, cudaStream_t s) {
     if (capacity == 0) return cudaSuccess;
-    gather_fp8_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
-        static_cast<const uint4*>(x), sorted_ids, offsets, E, k, H / 8, capacity, amax_bits,
-        static_cast<uint2*>(x_perm));
-    return cudaGetLastError();
+    return launch_pdl(gather_fp8_kernel, dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock),
+                      dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
+                      k, H / 8, capacity, amax_bits, static_cast<uint2*>(x_perm));
 }
 
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
                                   int capacity, const uint32_t* amax_bits, void* h_q,
                                   cudaStream_t s) {
     if (capacity == 0) return cudaSuccess;
-    quant_rows_fp8_kernel<<<(capacity + kRowsPerBlock - 1) / kRowsPerBlock, kThreads, 0, s>>>(
-        static_cast<const uint4*>(h), offsets, E, cols / 8, capacity, amax_bits,
-        static_cast<uint2*>(h_q));
-    return cudaGetLastError();
+    return launch_pdl(quant_rows_fp8_kernel, dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock),
+                      dim3(kThreads), 0, s, static_cast<const uint4*>(h), offsets, E, cols / 8,
+                      capacity, amax_bits, static_cast<uint2*>(h_q));
 }
 
 cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
                            void* out, cudaStream_t s) {
     const long n = static_cast<long>(T) * (H / 8);
     if (n == 0) return cudaSuccess;
-    combine_kernel<<<static_cast<unsigned>((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(
-        static_cast<const uint4*>(y_perm), inv_perm, T, k, H / 8, static_cast<uint4*>(out));
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(static_cast<unsigned>((n + kThreads - 1) / kThreads)),
+                      dim3(kThreads), 0, s, static_cast<const uint4*>(y_perm), inv_perm, T, k,
+                      H / 8, static_cast<uint4*>(out));
 }
 
 cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, const void* Wu,
@@ -288,17 +291,20 @@ cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, co
     const auto* u = static_cast<const __nv_bfloat16*>(Wu);
     const auto* d = static_cast<const __nv_bfloat16*>(Wd);
     const long hi = static_cast<long>(H) * I;
-    const long elt = fp8 ? 1 : 2;
+    const PackedGeom geo = packed_geom(fp8, E, H, I);
+    uint8_t* gu = static_cast<uint8_t*>(packed);
+    uint8_t* dn = gu + geo.gu_bytes;
+    const dim3 ggu(geo.kb_gu, geo.mt_gu, E), gdn(geo.kb_dn, geo.mt_dn, E);
     if (fp8) {
         cudaError_t err = cudaMemsetAsync(amax_tmp, 0, sizeof(uint32_t) * 3 * E, s);
         if (err != cudaSuccess) return err;
         matrix_amax_kernel<<<dim3(blocks_for(hi / 8, kThreads * 8, 64), 3 * E), kThreads, 0, s>>>(
             reinterpret_cast<const uint4*>(g), reinterpret_cast<const uint4*>(u),
             reinterpret_cast<const uint4*>(d), hi / 8, amax_tmp);
-        pack_gate_up_kernel<true><<<dim3(2 * I / 32, H / 64, E), kThreads, 0, s>>>(g, u, H, I,
-                                                                                  packed, amax_tmp);
-        pack_down_kernel<true><<<dim3(H / 32, I / 32, E), kThreads, 0, s>>>(
-            d, H, I, packed, 2 * static_cast<long>(E) * hi, amax_tmp);
+        pack_tiles_kernel<true, true><<<ggu, kThreads, 0, s>>>(g, u, H, I, geo.mt_gu, geo.kb_gu,
+                                                               gu, amax_tmp);
+        pack_tiles_kernel<true, false><<<gdn, kThreads, 0, s>>>(d, nullptr, H, I, geo.mt_dn,
+                                                                geo.kb_dn, dn, amax_tmp);
         if (static_cast<void*>(scales) != static_cast<void*>(amax_tmp)) {
             err = cudaMemcpyAsync(scales, amax_tmp, sizeof(float) * 3 * E, cudaMemcpyDeviceToDevice,
                                   s);
@@ -306,12 +312,11 @@ cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, co
         }
         amax_to_scale_kernel<<<(3 * E + 255) / 256, 256, 0, s>>>(scales, 3 * E);
     } else {
-        pack_gate_up_kernel<false><<<dim3(2 * I / 32, H / 64, E), kThreads, 0, s>>>(
-            g, u, H, I, packed, nullptr);
-        pack_down_kernel<false><<<dim3(H / 32, I / 32, E), kThreads, 0, s>>>(
-            d, H, I, packed, 2 * static_cast<long>(E) * hi, nullptr);
+        pack_tiles_kernel<false, true><<<ggu, kThreads, 0, s>>>(g, u, H, I, geo.mt_gu, geo.kb_gu,
+                                                                gu, nullptr);
+        pack_tiles_kernel<false, false><<<gdn, kThreads, 0, s>>>(d, nullptr, H, I, geo.mt_dn,
+                                                                 geo.kb_dn, dn, nullptr);
     }
-    (void)elt;
     return cudaGetLastError();
 }
 

@@ -25,6 +25,14 @@
 // accumulators of nmax fp32 columns so the epilogue of one unit overlaps the
 // main loop of the next.  Every wait is bounded; on expiry the kernel records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+//
+// Weights (A) are pre-packed as 16 KB tiles that are already the swizzled
+// shared-memory image of one stage, so each stage's A operand is one
+// contiguous bulk copy and a CTA's stream-K range is one sequential stream
+// through memory.  Activations (B) come through TMA tensor maps with 64-row
+// and 16-row boxes, so a token tile moves only its own rows.  Launched with
+// programmatic dependent launch: the producer fetches the first weight tiles
+// before waiting for the previous kernel, whose output (B) it loads after.
 #include <mutex>
 
 #include "common.cuh"
@@ -47,7 +55,8 @@ constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
 struct GemmArgs {
     int E, Mw, K, KB, MT, Mvalid;
-    int nmax, box_rows, stages, tmem_cols;
+    int nmax, stages, kps, tmem_cols;
+    const uint8_t* a_tiles;
     int ldo;
     void* out;
     const int32_t* counts;
@@ -84,6 +93,8 @@ struct Ctl {
 struct Seg {
     int u, kb0, kb1, e, m, b_row, N;
 };
+
+constexpr int kDynSmemMax = kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024;
 
 __device__ __forceinline__ int find_expert(const int* prefix, int E, int u) {
     int lo = 0, hi = E - 1;
@@ -167,8 +178,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
         }
         float wt = 0.0f;
         if (lane < 16) {
-            const int sid = g.sorted_ids[s.b_row + c0 + lane];
-            wt = sid >= 0 ? g.route_w[sid] : 0.0f;
+            const int sid = __ldcg(g.sorted_ids + s.b_row + c0 + lane);
+            wt = sid >= 0 ? __ldcg(g.route_w + sid) : 0.0f;
         }
         __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + wq * 1024);
 #pragma unroll
@@ -195,26 +206,31 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
 
 template <bool FP8, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB64,
+                        const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ Ctl ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // stage = kps consecutive k-blocks: A kps*16 KB (one bulk copy), B kps
+    // slots of nmax rows x 128 B
+    const int KPS = g.kps;
+    const int a_stage_bytes = KPS * kATileBytes;
+    const int b_kb_bytes = g.nmax * kRowBytes;
+    const int b_stage_bytes = KPS * b_kb_bytes;
     uint8_t* smA = base;
-    uint8_t* smB = smA + g.stages * kATileBytes;
-    uint8_t* staging = smB + g.stages * g.nmax * kRowBytes;
-    const int b_stage_bytes = g.nmax * kRowBytes;
+    uint8_t* smB = smA + g.stages * a_stage_bytes;
+    uint8_t* staging = smB + g.stages * b_stage_bytes;
 
     // ---- schedule tables: per-expert counts, offsets, token tiles, unit prefix
     {
         const int e = threadIdx.x;
         int units = 0;
         if (e < g.E) {
-            const int c = g.counts[e];
+            const int c = __ldcg(g.counts + e);
             ctl.cnt[e] = c;
-            ctl.off[e] = g.offsets[e];
+            ctl.off[e] = __ldcg(g.offsets + e);
             const int nt = (c + g.nmax - 1) / g.nmax;
             ctl.ntt[e] = nt;
             units = nt * g.MT;
@@ -243,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl.mma_issued = 0;
         }
         if (warp == 0 && lane == 0) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmB64);
+            tma_prefetch_desc(&tmB16);
         }
         if (warp == 2) {
             tmem_alloc(&ctl.tmem_base, g.tmem_cols);
@@ -281,35 +297,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0 && active) {
+        if (lane == 0) {
             uint32_t it = 0;
             const int bk_elems = FP8 ? 128 : 64;
-            for (long long x = ws; x < we;) {
-                const Seg s = make_seg(ctl, g, x, we);
-                const int a_row = s.e * g.Mw + s.m * kBM;
-                const int nload = (s.N + g.box_rows - 1) / g.box_rows;
-                const uint32_t bytes = kATileBytes + nload * g.box_rows * kRowBytes;
-                bool ok = true;
-                for (int kb = s.kb0; kb < s.kb1; ++kb, ++it) {
-                    const int st = it % S;
-                    const uint32_t par = ((it / S) & 1u) ^ 1u;
-                    if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
-                        raise_abort(ctl, g.status);
-                        ok = false;
-                        break;
+            // Stages whose weight tiles are issued before the wait for the
+            // previous kernel; their activation rows follow after it.
+            int early = 0;
+            if (active) {
+                for (long long x = ws; x < we && early < S;) {
+                    const Seg s = make_seg(ctl, g, x, we);
+                    const uint8_t* a = g.a_tiles +
+                                       (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
+                    const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
+                    for (int kb = s.kb0; kb < s.kb1 && early < S; kb += KPS, ++early) {
+                        const int nk = min(KPS, s.kb1 - kb);
+                        mbar_arrive_expect_tx(&ctl.full[early],
+                                              nk * (kATileBytes + (n64 * 64 + n16 * 16) * kRowBytes));
+                        bulk_load(smA + early * a_stage_bytes,
+                                  a + static_cast<size_t>(kb) * kTileBytes, nk * kATileBytes,
+                                  &ctl.full[early], kEvictFirst);
                     }
-                    mbar_arrive_expect_tx(&ctl.full[st], bytes);
-                    tma_load_2d(smA + st * kATileBytes, &tmA, &ctl.full[st], kb * bk_elems, a_row,
-                                kEvictFirst);
-                    for (int j = 0; j < nload; ++j)
-                        tma_load_2d(smB + st * b_stage_bytes + j * g.box_rows * kRowBytes, &tmB,
-                                    &ctl.full[st], kb * bk_elems, s.b_row + j * g.box_rows,
-                                    kEvictLast);
+                    x += s.kb1 - s.kb0;
+                }
+            }
+            pdl_wait();
+            pdl_trigger();
+            for (long long x = ws; active && x < we;) {
+                const Seg s = make_seg(ctl, g, x, we);
+                const uint8_t* a = g.a_tiles +
+                                   (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
+                const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
+                const uint32_t kb_bytes = kATileBytes + (n64 * 64 + n16 * 16) * kRowBytes;
+                bool ok = true;
+                for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
+                    const int st = it % S;
+                    const int nk = min(KPS, s.kb1 - kb);
+                    if (it >= static_cast<uint32_t>(early)) {
+                        const uint32_t par = ((it / S) & 1u) ^ 1u;
+                        if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
+                            raise_abort(ctl, g.status);
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&ctl.full[st], nk * kb_bytes);
+                        bulk_load(smA + st * a_stage_bytes,
+                                  a + static_cast<size_t>(kb) * kTileBytes, nk * kATileBytes,
+                                  &ctl.full[st], kEvictFirst);
+                    }
+                    for (int q = 0; q < nk; ++q) {
+                        uint8_t* b = smB + st * b_stage_bytes + q * b_kb_bytes;
+                        int row = s.b_row;
+                        const int xk = (kb + q) * bk_elems;
+                        for (int j = 0; j < n64; ++j, row += 64, b += 64 * kRowBytes)
+                            tma_load_2d(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
+                        for (int j = 0; j < n16; ++j, row += 16, b += 16 * kRowBytes)
+                            tma_load_2d(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
+                    }
                 }
                 if (!ok) break;
                 x += s.kb1 - s.kb0;
             }
-            ctl.prod_pos = it;
+            ctl.prod_pos = it > static_cast<uint32_t>(early) ? it : static_cast<uint32_t>(early);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -327,20 +375,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * g.nmax;
                 const uint32_t idesc = make_idesc<FP8>(kBM, s.N);
-                for (int kb = s.kb0; kb < s.kb1; ++kb, ++it) {
+                for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
                     const int st = it % S;
+                    const int nk = min(KPS, s.kb1 - kb);
                     if (!mbar_wait(&ctl.full[st], (it / S) & 1u, &ctl.abort)) {
                         raise_abort(ctl, g.status);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = sw128_desc(smem_u32(smA + st * kATileBytes));
-                    const uint64_t bd = sw128_desc(smem_u32(smB + st * b_stage_bytes));
+                    for (int q = 0; q < nk; ++q) {
+                        const uint64_t ad =
+                            sw128_desc(smem_u32(smA + st * a_stage_bytes + q * kATileBytes));
+                        const uint64_t bd =
+                            sw128_desc(smem_u32(smB + st * b_stage_bytes + q * b_kb_bytes));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc,
-                                  (kb > s.kb0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc,
+                                      (kb > s.kb0 || q > 0 || kk > 0) ? 1u : 0u);
+                    }
                     ctl.mma_issued = 1;
                     umma_commit(&ctl.empty[st]);
                 }
@@ -356,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp - kEpiWarp0;
         const int row = 32 * wq + lane;  // accumulator row = TMEM lane
         float act_scale = 1.0f;
-        if constexpr (FP8) act_scale = fp8_scale_from_amax(*g.act_amax);
+        if constexpr (FP8) act_scale = fp8_scale_from_amax(__ldcg(g.act_amax));
         float amax = 0.0f;
         uint32_t si = 0;
         for (long long x = ws; active && x < we; ++si) {
@@ -470,6 +523,8 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int K, long rows, int box_rows) {
+    // Zero-size tensors are not encodable; a one-row placeholder is never read.
+    if (rows < 1) rows = 1;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -484,13 +539,16 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int K, long rows, int b
 }
 
 template <bool FP8, int EPI>
-cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+cudaError_t launch_t(const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& g, int grid,
                      int smem, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<FP8, EPI>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, smem, s>>>(a, b, g);
-    return cudaGetLastError();
+    // Every launch asks for at most kSmemCap - sizeof(Ctl) - 1024 bytes (see
+    // the stage count below); the 1 KB margin covers the compiler's padding
+    // of the static shared block.
+    static cudaError_t attr = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmemMax);
+    if (attr != cudaSuccess) return attr;
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, b64, b16, g);
 }
 
 int pow2_at_least(int v) {
@@ -508,10 +566,13 @@ int device_sm_count() {
     return n > kMaxCtas ? kMaxCtas : n;
 }
 
-int gemm_nmax_for(int T) {
-    int n = (T + 15) & ~15;
+int gemm_nmax_for(int T, int k, int E) {
+    // Twice the mean tokens per expert, in steps of 16 (16..256); experts with
+    // more tokens are split into several token tiles.
+    const long mean2 = (2L * T * k + E - 1) / E;
+    long n = (mean2 + 15) & ~15L;
     if (n < 16) n = 16;
-    return n > 256 ? 256 : n;
+    return static_cast<int>(n > 256 ? 256 : n);
 }
 
 size_t gemm_partials_bytes(int nmax) {
@@ -523,18 +584,23 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.E = p.E;
     g.Mw = p.Mw;
     g.K = p.K;
-    const int bk = p.fp8 ? 128 : 64;
-    g.KB = (p.K + bk - 1) / bk;
-    g.MT = (p.Mw + kBM - 1) / kBM;
     g.Mvalid = p.Mvalid;
     g.nmax = p.nmax;
-    g.box_rows = p.nmax < 64 ? p.nmax : 64;
-    const int stage_bytes = kATileBytes + p.nmax * kRowBytes;
-    int stages = (kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024 - kStagingBytes - 1024) /
-                 stage_bytes;
-    if (stages > kMaxStages) stages = kMaxStages;
+    g.KB = p.KB;
+    g.MT = p.MT;
+    g.a_tiles = static_cast<const uint8_t*>(p.weights);
+    // Weight streaming (small token tiles): 4 k-blocks per stage, i.e. 64 KB
+    // bulk copies, two stages (~128 KB in flight per SM) -- measured on B200
+    // to sustain a higher HBM read rate than more, smaller copies.  Large
+    // token tiles are tensor-bound and keep one k-block per stage.
+    const int kps = p.nmax <= 64 ? 4 : 1;
+    const int max_stages = p.nmax <= 64 ? 2 : kMaxStages;
+    const int stage_bytes = kps * (kATileBytes + p.nmax * kRowBytes);
+    int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
+    if (stages > max_stages) stages = max_stages;
     if (stages < 2) return cudaErrorInvalidValue;
     g.stages = stages;
+    g.kps = kps;
     g.tmem_cols = pow2_at_least(2 * p.nmax);
     g.ldo = p.ldo;
     g.out = p.out;
@@ -548,19 +614,19 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.partials = p.partials;
     g.counters = p.counters;
     g.status = p.status;
-    CUtensorMap ta, tb;
-    if (!make_map(&ta, p.weights, p.fp8, p.K, static_cast<long>(p.E) * p.Mw, kBM) ||
-        !make_map(&tb, p.act, p.fp8, p.K, p.capacity, g.box_rows))
+    CUtensorMap tb64, tb16;
+    if (!make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
+        !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16))
         return cudaErrorInvalidValue;
     int grid = device_sm_count();
     if (p.max_ctas > 0 && p.max_ctas < grid) grid = p.max_ctas;
     const int smem = 1024 + stages * stage_bytes + kStagingBytes;
     if (p.fp8) {
-        return p.epi == 0 ? launch_t<true, 0>(ta, tb, g, grid, smem, s)
-                          : launch_t<true, 1>(ta, tb, g, grid, smem, s);
+        return p.epi == 0 ? launch_t<true, 0>(tb64, tb16, g, grid, smem, s)
+                          : launch_t<true, 1>(tb64, tb16, g, grid, smem, s);
     }
-    return p.epi == 0 ? launch_t<false, 0>(ta, tb, g, grid, smem, s)
-                      : launch_t<false, 1>(ta, tb, g, grid, smem, s);
+    return p.epi == 0 ? launch_t<false, 0>(tb64, tb16, g, grid, smem, s)
+                      : launch_t<false, 1>(tb64, tb16, g, grid, smem, s);
 }
 
 }  // namespace moe

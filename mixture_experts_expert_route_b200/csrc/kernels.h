@@ -9,9 +9,55 @@
 
 namespace moe {
 
+// Packed expert weights are stored as 16 KB tiles, each the exact shared-memory
+// image (128-byte swizzle) of 128 weight rows x 128 bytes of K, so that one
+// contiguous bulk copy fills one pipeline stage.  Tile (m, kb) of expert e of a
+// matrix with MT row tiles and KB k-blocks lives at ((e*MT + m)*KB + kb)*16 KB.
+// Rows past the matrix and K past its length are zero.
+constexpr int kTileRows = 128;
+constexpr int kTileRowBytes = 128;
+constexpr int kTileBytes = kTileRows * kTileRowBytes;
+struct PackedGeom {
+    int bk;               // K elements per tile row (64 bf16, 128 e4m3)
+    int mt_gu, kb_gu;     // gate/up: 2I/128 row tiles, ceil(H/bk) k-blocks
+    int mt_dn, kb_dn;     // down: ceil(H/128) row tiles, ceil(I/bk) k-blocks
+    size_t gu_bytes;      // all experts
+    size_t dn_bytes;
+};
+inline PackedGeom packed_geom(int fp8, int E, int H, int I) {
+    PackedGeom g;
+    g.bk = fp8 ? 128 : 64;
+    g.mt_gu = (2 * I + kTileRows - 1) / kTileRows;
+    g.kb_gu = (H + g.bk - 1) / g.bk;
+    g.mt_dn = (H + kTileRows - 1) / kTileRows;
+    g.kb_dn = (I + g.bk - 1) / g.bk;
+    g.gu_bytes = static_cast<size_t>(E) * g.mt_gu * g.kb_gu * kTileBytes;
+    g.dn_bytes = static_cast<size_t>(E) * g.mt_dn * g.kb_dn * kTileBytes;
+    return g;
+}
+
+// Launch with programmatic dependent launch allowed (see pdl_wait/pdl_trigger).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- a1/a2 (route_permute.cu)
+// ctl (optional): the layer's control block, zeroed by the first kernel of a
+// forward call after it has waited for the previous call's kernels.
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                              cudaStream_t s);
+                              cudaStream_t s, int32_t* ctl = nullptr, int ctl_ints = 0);
 // Single-CTA route + permute for small batches (T <= kSmallT, T*k <= kChunk).
 constexpr int kSmallT = 128;
 constexpr int kChunk = 2048;  // assignments per permutation chunk
@@ -21,7 +67,7 @@ cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k,
                                        int capacity, int32_t* ids, float* w, int32_t* counts,
                                        int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
-                                       cudaStream_t s);
+                                       cudaStream_t s, int32_t* ctl = nullptr, int ctl_ints = 0);
 cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
                                  int capacity, int32_t* counts, int32_t* offsets,
                                  int32_t* sorted_ids, int32_t* inv_perm, int32_t* tiles,
@@ -53,7 +99,8 @@ struct GemmProblem {
     int Mvalid;           // weight rows per expert that are real (masking)
     int nmax;             // token-tile cap (multiple of 16, <= 256)
     int capacity;         // rows of the activation operand
-    const void* weights;  // packed [E*Mw, K]
+    const void* weights;  // packed tiles of this matrix (see PackedGeom)
+    int MT, KB;           // row tiles and k-blocks per expert
     const void* act;      // [capacity, K]
     void* out;            // [capacity, ldo] bf16
     int ldo;
@@ -69,7 +116,7 @@ struct GemmProblem {
     int32_t* status;
     int max_ctas;
 };
-int gemm_nmax_for(int T);
+int gemm_nmax_for(int T, int k, int E);
 size_t gemm_partials_bytes(int nmax);
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 

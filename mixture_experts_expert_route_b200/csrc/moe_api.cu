@@ -103,7 +103,7 @@ void record(moe_event_t* ev, int i, cudaStream_t s) {
 // a3..a6 on carved buffers.  The control block must already be zeroed.
 moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaStream_t s) {
     const bool fp8 = f.dt == MOE_FP8_E4M3;
-    const int nmax = gemm_nmax_for(f.T);
+    const int nmax = gemm_nmax_for(f.T, f.k, f.E);
     uint32_t* amax_x = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxX);
     uint32_t* amax_h = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxH);
     cudaError_t e;
@@ -118,7 +118,7 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 2, s);
 
-    const size_t elt = fp8 ? 1 : 2;
+    const PackedGeom geo = packed_geom(fp8, f.E, f.H, f.I);
     GemmProblem gu{};
     gu.fp8 = fp8;
     gu.epi = 0;
@@ -129,6 +129,8 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     gu.nmax = nmax;
     gu.capacity = f.cap;
     gu.weights = f.packed;
+    gu.MT = geo.mt_gu;
+    gu.KB = geo.kb_gu;
     gu.act = b.x_perm;
     gu.out = b.h;
     gu.ldo = f.I;
@@ -154,7 +156,9 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     dn.Mw = f.H;
     dn.K = f.I;
     dn.Mvalid = f.H;
-    dn.weights = static_cast<const char*>(f.packed) + 2 * static_cast<size_t>(f.E) * f.H * f.I * elt;
+    dn.weights = static_cast<const char*>(f.packed) + geo.gu_bytes;
+    dn.MT = geo.mt_dn;
+    dn.KB = geo.kb_dn;
     dn.act = fp8 ? b.h_q : b.h;
     dn.out = f.y_perm;
     dn.ldo = f.H;
@@ -171,7 +175,7 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
 size_t ffn_ws_bytes(moe_dtype dt, int T, int k, int E, int H, int I, int block_m) {
     Carver c{nullptr};
     const int cap = moe_permute_capacity(T, k, E, block_m);
-    carve_ffn(c, dt, cap, H, I, gemm_nmax_for(T));
+    carve_ffn(c, dt, cap, H, I, gemm_nmax_for(T, k, E));
     return c.used;
 }
 
@@ -204,7 +208,7 @@ FwdBuffers carve_fwd(Carver& c, moe_dtype dt, int T, int k, int E, int H, int I,
     b.tiles = c.take<int32_t>(sizeof(int32_t) * (cap / block_m + 1));
     b.chunk_counts = c.take<int32_t>(sizeof(int32_t) * permute_chunks(A) * E);
     b.y_perm = c.take<void>(static_cast<size_t>(cap) * H * 2);
-    carve_ffn_rest(c, b.ffn, dt, cap, H, I, gemm_nmax_for(T));
+    carve_ffn_rest(c, b.ffn, dt, cap, H, I, gemm_nmax_for(T, k, E));
     return b;
 }
 
@@ -275,8 +279,8 @@ moe_status moe_align_permute(const int32_t* ids, int T, int k, int E, int block_
 
 size_t moe_packed_weights_size(moe_dtype dtype, int E, int H, int I) {
     if (E < 1 || H < 1 || I < 1) return 0;
-    const size_t elt = dtype == MOE_FP8_E4M3 ? 1 : 2;
-    return 3 * static_cast<size_t>(E) * H * I * elt;
+    const PackedGeom g = packed_geom(dtype == MOE_FP8_E4M3, E, H, I);
+    return g.gu_bytes + g.dn_bytes;
 }
 
 moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const void* Wg, const void* Wu,
@@ -317,7 +321,7 @@ moe_status moe_grouped_ffn(const moe_ffn_args* a, void* ws, size_t ws_bytes, moe
     if (!ws || ws_bytes < need_ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     Carver c{static_cast<char*>(ws)};
-    const FfnBuffers b = carve_ffn(c, a->dtype, a->capacity, a->H, a->I, gemm_nmax_for(a->T));
+    const FfnBuffers b = carve_ffn(c, a->dtype, a->capacity, a->H, a->I, gemm_nmax_for(a->T, a->k, a->E));
     if (cudaMemsetAsync(b.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, a->capacity, a->x, a->w, a->counts,
@@ -371,15 +375,16 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     moe_event_t* ev = a->events;
 
     record(ev, 0, s);
-    if (cudaMemsetAsync(b.ffn.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    // The first kernel zeroes the control block (counters, amax words, and
+    // the status word when the caller gave none) once the previous call's
+    // kernels are done with it.
     cudaError_t e;
     if (fused_route_permute_ok(a->T, a->k)) {
         e = launch_route_permute_small(a->logits, a->T, a->E, a->k, block_m, cap, ids, w, b.counts,
                                        b.offsets, b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,
-                                       status, s);
+                                       status, s, b.ffn.ctl, kCtlInts);
     } else {
-        e = launch_route_topk(a->logits, a->T, a->E, a->k, ids, w, s);
+        e = launch_route_topk(a->logits, a->T, a->E, a->k, ids, w, s, b.ffn.ctl, kCtlInts);
         if (e == cudaSuccess)
             e = launch_align_permute(ids, a->T, a->k, a->E, block_m, cap, b.counts, b.offsets,
                                      b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,

@@ -9,7 +9,7 @@
 // a2: the "data reordering" of "Az AWS új MoE-optimalizációkkal gyorsítja a
 //     SageMaker AI-t", § "A fused MoE a számítási folyamat több lépését
 //     egyesíti": a stable counting sort of the assignments by expert, with no
-//     atomics.  Assignments are cut into chunks of 2048 (256 per warp); each
+//     atomics.  Assignments are cut into chunks of 2048 (a slice per warp); each
 //     warp counts its slice with __match_any_sync (the lowest lane of each
 //     group of equal ids adds the group size to the warp's private histogram),
 //     per-expert prefix sums over (chunk, warp) give every warp a start
@@ -26,9 +26,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kPerWarp = kChunk / kWarps;  // 256 assignments per warp per chunk
+constexpr int kThreads = 256;        // multi-CTA kernels: 8 warps
+constexpr int kSmallThreads = 512;   // single-CTA kernel: 16 warps
+constexpr int kStageFloats = 4096;   // logits staged in smem by the single-CTA kernel
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ bool beats(float a, int ia, float b, int ib) {
@@ -41,10 +41,11 @@ __device__ __forceinline__ bool beats(float a, int ia, float b, int ib) {
     return ia < ib;
 }
 
-// Top-k of row[0..E) by one warp; sel is this warp's scratch of >= k floats.
+// Top-k of row[0..E) by one warp (row in global or shared memory).  Lane 0
+// writes the ids in selection order; the weights are a softmax over the
+// selected logits, re-read through the ids.
 template <int EPL>
-__device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                          float* __restrict__ w, float* sel) {
+__device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w) {
     const int lane = threadIdx.x & 31;
     float v[EPL];
     uint32_t taken = 0;
@@ -54,6 +55,7 @@ __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* 
         v[i] = e < E ? row[e] : 0.0f;
         if (e >= E) taken |= 1u << i;
     }
+    float m = 0.0f;
     for (int j = 0; j < k; ++j) {
         float bv = 0.0f;
         int bi = INT_MAX;
@@ -76,36 +78,40 @@ __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* 
             }
         }
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == 0) {
-            ids[j] = bi;
-            sel[j] = bv;
-        }
+        if (lane == 0) ids[j] = bi;
+        if (j == 0) m = bv;
     }
     __syncwarp();
-    const float m = sel[0];
     float z = 0.0f;
-    for (int j = lane; j < k; j += 32) z += expf(sel[j] - m);
+    for (int j = lane; j < k; j += 32) z += expf(row[ids[j]] - m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
-    for (int j = lane; j < k; j += 32) w[j] = expf(sel[j] - m) / z;
+    for (int j = lane; j < k; j += 32) w[j] = expf(row[ids[j]] - m) / z;
     __syncwarp();
+}
+
+__device__ void zero_ctl(int32_t* ctl, int n, int tid, int nthreads) {
+    for (int i = tid; i < n; i += nthreads) ctl[i] = 0;
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(kThreads) route_topk_kernel(const float* __restrict__ logits,
-                                                              int T, int E, int k,
-                                                              int32_t* __restrict__ ids,
-                                                              float* __restrict__ w) {
-    __shared__ float sel[kWarps][kMaxExperts];
+__global__ void __launch_bounds__(kThreads)
+    route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* ids,
+                      float* w, int32_t* ctl, int ctl_ints) {
+    pdl_wait();
+    pdl_trigger();
+    if (blockIdx.x == 0 && ctl) zero_ctl(ctl, ctl_ints, threadIdx.x, kThreads);
     const int warp = threadIdx.x >> 5;
-    const long t = static_cast<long>(blockIdx.x) * kWarps + warp;
+    const long t = static_cast<long>(blockIdx.x) * (kThreads / 32) + warp;
     if (t >= T) return;
-    warp_topk<EPL>(logits + t * E, E, k, ids + t * k, w + t * k, sel[warp]);
+    warp_topk<EPL>(logits + t * E, E, k, ids + t * k, w + t * k);
 }
 
 // hist[w][e] += number of assignments of warp w's slice of the chunk routed to e
-__device__ void chunk_histogram(const int32_t* __restrict__ ids, long A, long chunk_base, int E,
+template <int NW>
+__device__ void chunk_histogram(const int32_t* ids, long A, long chunk_base, int E,
                                 int (*hist)[kMaxExperts], int32_t* status) {
+    constexpr int kPerWarp = kChunk / NW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long wbase = chunk_base + static_cast<long>(warp) * kPerWarp;
     for (int r = 0; r < kPerWarp / 32; ++r) {
@@ -125,9 +131,10 @@ __device__ void chunk_histogram(const int32_t* __restrict__ ids, long A, long ch
 }
 
 // Places the warp's slice: base[w][e] holds the next free slot of expert e.
-__device__ void chunk_scatter(const int32_t* __restrict__ ids, long A, long chunk_base, int E,
-                              int (*base)[kMaxExperts], int32_t* __restrict__ sorted_ids,
-                              int32_t* __restrict__ inv_perm) {
+template <int NW>
+__device__ void chunk_scatter(const int32_t* ids, long A, long chunk_base, int E,
+                              int (*base)[kMaxExperts], int32_t* sorted_ids, int32_t* inv_perm) {
+    constexpr int kPerWarp = kChunk / NW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long wbase = chunk_base + static_cast<long>(warp) * kPerWarp;
     for (int r = 0; r < kPerWarp / 32; ++r) {
@@ -149,8 +156,10 @@ __device__ void chunk_scatter(const int32_t* __restrict__ ids, long A, long chun
     }
 }
 
-// Exclusive scan over the 256 threads of the block.
-__device__ int block_exclusive_scan(int v, int* tmp /* kWarps + 1 */) {
+// Exclusive scan of one value per thread over the NT threads of the block.
+template <int NT>
+__device__ int block_exclusive_scan(int v, int* tmp /* NT/32 + 1 */) {
+    constexpr int NW = NT / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int inc = v;
 #pragma unroll
@@ -162,12 +171,12 @@ __device__ int block_exclusive_scan(int v, int* tmp /* kWarps + 1 */) {
     __syncthreads();
     if (threadIdx.x == 0) {
         int run = 0;
-        for (int i = 0; i < kWarps; ++i) {
+        for (int i = 0; i < NW; ++i) {
             const int t = tmp[i];
             tmp[i] = run;
             run += t;
         }
-        tmp[kWarps] = run;
+        tmp[NW] = run;
     }
     __syncthreads();
     return tmp[warp] + inc - v;
@@ -175,12 +184,13 @@ __device__ int block_exclusive_scan(int v, int* tmp /* kWarps + 1 */) {
 
 // Thread e < E: given the total count c of expert e, writes counts, offsets,
 // tiles and the pads of e's block; returns o_e.  All threads must call it.
+template <int NT>
 __device__ int finish_offsets(int c, int E, int block_m, int32_t* counts, int32_t* offsets,
                               int32_t* sorted_ids, int32_t* tiles, int32_t* num_tiles,
                               int* tmp) {
     const int e = threadIdx.x;
     const int padded = (e < E) ? (c + block_m - 1) / block_m * block_m : 0;
-    const int o = block_exclusive_scan(padded, tmp);
+    const int o = block_exclusive_scan<NT>(padded, tmp);
     if (e < E) {
         counts[e] = c;
         offsets[e] = o;
@@ -194,65 +204,82 @@ __device__ int finish_offsets(int c, int E, int block_m, int32_t* counts, int32_
     return o;
 }
 
+template <int NT>
 __device__ void fill_tail(int total, int block_m, int capacity, int32_t* sorted_ids,
                           int32_t* tiles) {
-    for (int p = total + threadIdx.x; p < capacity; p += kThreads) sorted_ids[p] = -1;
-    for (int b = total / block_m + threadIdx.x; b < capacity / block_m; b += kThreads)
-        tiles[b] = -1;
+    for (int p = total + threadIdx.x; p < capacity; p += NT) sorted_ids[p] = -1;
+    for (int b = total / block_m + threadIdx.x; b < capacity / block_m; b += NT) tiles[b] = -1;
 }
 
-// One CTA: optional routing of all T tokens, then the whole permutation of
-// A = T*k <= kChunk assignments.
+// One CTA of 16 warps: optional routing of all T tokens (logits staged in
+// shared memory when they fit), then the whole permutation of A = T*k <=
+// kChunk assignments.
 template <int EPL>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kSmallThreads)
     route_permute_small_kernel(const float* __restrict__ logits, int T, int E, int k, int block_m,
                                int capacity, int32_t* ids, float* w, int32_t* counts,
                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
-                               int32_t* tiles, int32_t* num_tiles, int32_t* status) {
-    __shared__ int hist[kWarps][kMaxExperts];
-    __shared__ float sel[kWarps][kMaxExperts];
-    __shared__ int tmp[kWarps + 1];
+                               int32_t* tiles, int32_t* num_tiles, int32_t* status, int32_t* ctl,
+                               int ctl_ints) {
+    constexpr int NW = kSmallThreads / 32;
+    __shared__ int hist[NW][kMaxExperts];
+    __shared__ float slog[kStageFloats];
+    __shared__ int tmp[NW + 1];
     const int warp = threadIdx.x >> 5;
     const long A = static_cast<long>(T) * k;
+    pdl_wait();
+    pdl_trigger();
+    if (ctl) zero_ctl(ctl, ctl_ints, threadIdx.x, kSmallThreads);
     if (logits) {
-        for (int t = warp; t < T; t += kWarps)
-            warp_topk<EPL>(logits + static_cast<long>(t) * E, E, k, ids + static_cast<long>(t) * k,
-                           w + static_cast<long>(t) * k, sel[warp]);
+        const int n = T * E;
+        const float* src = logits;
+        if (n <= kStageFloats) {
+            for (int i = threadIdx.x; i < n; i += kSmallThreads) slog[i] = logits[i];
+            __syncthreads();
+            src = slog;
+        }
+        for (int t = warp; t < T; t += NW)
+            warp_topk<EPL>(src + static_cast<long>(t) * E, E, k, ids + static_cast<long>(t) * k,
+                           w + static_cast<long>(t) * k);
     }
-    for (int i = threadIdx.x; i < kWarps * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
+    for (int i = threadIdx.x; i < NW * kMaxExperts; i += kSmallThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    chunk_histogram(ids, A, 0, E, hist, status);
+    chunk_histogram<NW>(ids, A, 0, E, hist, status);
     __syncthreads();
     const int e = threadIdx.x;
     int c = 0;
     if (e < E)
-        for (int wq = 0; wq < kWarps; ++wq) c += hist[wq][e];
-    const int o = finish_offsets(c, E, block_m, counts, offsets, sorted_ids, tiles, num_tiles, tmp);
+        for (int wq = 0; wq < NW; ++wq) c += hist[wq][e];
+    const int o = finish_offsets<kSmallThreads>(c, E, block_m, counts, offsets, sorted_ids, tiles,
+                                                num_tiles, tmp);
     if (e < E) {
         int run = o;
-        for (int wq = 0; wq < kWarps; ++wq) {
+        for (int wq = 0; wq < NW; ++wq) {
             const int h = hist[wq][e];
             hist[wq][e] = run;
             run += h;
         }
     }
-    const int total = tmp[kWarps];
+    const int total = tmp[NW];
     __syncthreads();
-    fill_tail(total, block_m, capacity, sorted_ids, tiles);
-    chunk_scatter(ids, A, 0, E, hist, sorted_ids, inv_perm);
+    fill_tail<kSmallThreads>(total, block_m, capacity, sorted_ids, tiles);
+    chunk_scatter<NW>(ids, A, 0, E, hist, sorted_ids, inv_perm);
 }
 
 __global__ void __launch_bounds__(kThreads)
-    permute_count_kernel(const int32_t* __restrict__ ids, long A, int E,
-                         int32_t* __restrict__ chunk_counts, int32_t* status) {
-    __shared__ int hist[kWarps][kMaxExperts];
-    for (int i = threadIdx.x; i < kWarps * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
+    permute_count_kernel(const int32_t* ids, long A, int E, int32_t* __restrict__ chunk_counts,
+                         int32_t* status) {
+    constexpr int NW = kThreads / 32;
+    __shared__ int hist[NW][kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < NW * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    chunk_histogram(ids, A, static_cast<long>(blockIdx.x) * kChunk, E, hist, status);
+    chunk_histogram<NW>(ids, A, static_cast<long>(blockIdx.x) * kChunk, E, hist, status);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int c = 0;
-        for (int wq = 0; wq < kWarps; ++wq) c += hist[wq][e];
+        for (int wq = 0; wq < NW; ++wq) c += hist[wq][e];
         chunk_counts[static_cast<long>(blockIdx.x) * E + e] = c;
     }
 }
@@ -261,7 +288,10 @@ __global__ void __launch_bounds__(kThreads)
     permute_scan_kernel(int nchunks, int E, int block_m, int capacity, int32_t* chunk_counts,
                         int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* tiles,
                         int32_t* num_tiles) {
-    __shared__ int tmp[kWarps + 1];
+    constexpr int NW = kThreads / 32;
+    __shared__ int tmp[NW + 1];
+    pdl_wait();
+    pdl_trigger();
     const int e = threadIdx.x;
     int run = 0;
     if (e < E)
@@ -270,33 +300,36 @@ __global__ void __launch_bounds__(kThreads)
             chunk_counts[static_cast<long>(c) * E + e] = run;
             run += v;
         }
-    finish_offsets(run, E, block_m, counts, offsets, sorted_ids, tiles, num_tiles, tmp);
-    const int total = tmp[kWarps];
+    finish_offsets<kThreads>(run, E, block_m, counts, offsets, sorted_ids, tiles, num_tiles, tmp);
+    const int total = tmp[NW];
     __syncthreads();
-    fill_tail(total, block_m, capacity, sorted_ids, tiles);
+    fill_tail<kThreads>(total, block_m, capacity, sorted_ids, tiles);
 }
 
 __global__ void __launch_bounds__(kThreads)
-    permute_scatter_kernel(const int32_t* __restrict__ ids, long A, int E,
+    permute_scatter_kernel(const int32_t* ids, long A, int E,
                            const int32_t* __restrict__ chunk_prefix,
                            const int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
                            int32_t* __restrict__ inv_perm) {
-    __shared__ int hist[kWarps][kMaxExperts];
-    for (int i = threadIdx.x; i < kWarps * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
+    constexpr int NW = kThreads / 32;
+    __shared__ int hist[NW][kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < NW * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
     const long base = static_cast<long>(blockIdx.x) * kChunk;
-    chunk_histogram(ids, A, base, E, hist, nullptr);
+    chunk_histogram<NW>(ids, A, base, E, hist, nullptr);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int run = offsets[e] + chunk_prefix[static_cast<long>(blockIdx.x) * E + e];
-        for (int wq = 0; wq < kWarps; ++wq) {
+        for (int wq = 0; wq < NW; ++wq) {
             const int h = hist[wq][e];
             hist[wq][e] = run;
             run += h;
         }
     }
     __syncthreads();
-    chunk_scatter(ids, A, base, E, hist, sorted_ids, inv_perm);
+    chunk_scatter<NW>(ids, A, base, E, hist, sorted_ids, inv_perm);
 }
 
 int epl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
@@ -310,35 +343,33 @@ bool fused_route_permute_ok(int T, int k) {
 }
 
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                              cudaStream_t s) {
+                              cudaStream_t s, int32_t* ctl, int ctl_ints) {
     if (T == 0) return cudaSuccess;
-    const dim3 grid((T + kWarps - 1) / kWarps);
+    const dim3 grid((T + kThreads / 32 - 1) / (kThreads / 32));
     switch (epl_for(E)) {
-        case 1: route_topk_kernel<1><<<grid, kThreads, 0, s>>>(logits, T, E, k, ids, w); break;
-        case 2: route_topk_kernel<2><<<grid, kThreads, 0, s>>>(logits, T, E, k, ids, w); break;
-        case 4: route_topk_kernel<4><<<grid, kThreads, 0, s>>>(logits, T, E, k, ids, w); break;
-        default: route_topk_kernel<8><<<grid, kThreads, 0, s>>>(logits, T, E, k, ids, w); break;
+        case 1: return launch_pdl(route_topk_kernel<1>, grid, dim3(kThreads), 0, s, logits, T, E, k, ids, w, ctl, ctl_ints);
+        case 2: return launch_pdl(route_topk_kernel<2>, grid, dim3(kThreads), 0, s, logits, T, E, k, ids, w, ctl, ctl_ints);
+        case 4: return launch_pdl(route_topk_kernel<4>, grid, dim3(kThreads), 0, s, logits, T, E, k, ids, w, ctl, ctl_ints);
+        default: return launch_pdl(route_topk_kernel<8>, grid, dim3(kThreads), 0, s, logits, T, E, k, ids, w, ctl, ctl_ints);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k, int block_m,
                                        int capacity, int32_t* ids, float* w, int32_t* counts,
                                        int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
-                                       cudaStream_t s) {
-#define MOE_SMALL(EPL)                                                                          \
-    route_permute_small_kernel<EPL><<<1, kThreads, 0, s>>>(logits, T, E, k, block_m, capacity, \
-                                                           ids, w, counts, offsets, sorted_ids, \
-                                                           inv_perm, tiles, num_tiles, status)
+                                       cudaStream_t s, int32_t* ctl, int ctl_ints) {
+#define MOE_SMALL(EPL)                                                                            \
+    return launch_pdl(route_permute_small_kernel<EPL>, dim3(1), dim3(kSmallThreads), 0, s, logits, \
+                      T, E, k, block_m, capacity, ids, w, counts, offsets, sorted_ids, inv_perm,  \
+                      tiles, num_tiles, status, ctl, ctl_ints)
     switch (epl_for(E)) {
-        case 1: MOE_SMALL(1); break;
-        case 2: MOE_SMALL(2); break;
-        case 4: MOE_SMALL(4); break;
-        default: MOE_SMALL(8); break;
+        case 1: MOE_SMALL(1);
+        case 2: MOE_SMALL(2);
+        case 4: MOE_SMALL(4);
+        default: MOE_SMALL(8);
     }
 #undef MOE_SMALL
-    return cudaGetLastError();
 }
 
 cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
@@ -351,13 +382,18 @@ cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int bl
     if (nch <= 1)
         return launch_route_permute_small(nullptr, T, E, k, block_m, capacity,
                                           const_cast<int32_t*>(ids), nullptr, counts, offsets,
-                                          sorted_ids, inv_perm, tiles, num_tiles, status, s);
-    permute_count_kernel<<<nch, kThreads, 0, s>>>(ids, A, E, chunk_counts, status);
-    permute_scan_kernel<<<1, kThreads, 0, s>>>(nch, E, block_m, capacity, chunk_counts, counts,
-                                               offsets, sorted_ids, tiles, num_tiles);
-    permute_scatter_kernel<<<nch, kThreads, 0, s>>>(ids, A, E, chunk_counts, offsets, sorted_ids,
-                                                    inv_perm);
-    return cudaGetLastError();
+                                          sorted_ids, inv_perm, tiles, num_tiles, status, s,
+                                          nullptr, 0);
+    cudaError_t e = launch_pdl(permute_count_kernel, dim3(nch), dim3(kThreads), 0, s, ids, A, E,
+                               chunk_counts, status);
+    if (e == cudaSuccess)
+        e = launch_pdl(permute_scan_kernel, dim3(1), dim3(kThreads), 0, s, nch, E, block_m,
+                       capacity, chunk_counts, counts, offsets, sorted_ids, tiles, num_tiles);
+    if (e == cudaSuccess)
+        e = launch_pdl(permute_scatter_kernel, dim3(nch), dim3(kThreads), 0, s, ids, A, E,
+                       static_cast<const int32_t*>(chunk_counts),
+                       static_cast<const int32_t*>(offsets), sorted_ids, inv_perm);
+    return e;
 }
 
 }  // namespace moe

@@ -54,8 +54,10 @@ def test_workspace_sizes(L):
     lib = L.lib()
     assert lib.moe_align_permute_workspace_size(64, 2, 8) == 0       # single chunk
     assert lib.moe_align_permute_workspace_size(4096, 8, 128) == 16 * 128 * 4
+    # 16 KB tiles of 128 rows x 128 bytes, padded per expert matrix
     assert lib.moe_packed_weights_size(0, 8, 4096, 14336) == 3 * 8 * 4096 * 14336 * 2
-    assert lib.moe_packed_weights_size(1, 32, 2880, 2880) == 3 * 32 * 2880 * 2880
+    tiles = 32 * ((2 * 2880 // 128) * 23 + 23 * 23)
+    assert lib.moe_packed_weights_size(1, 32, 2880, 2880) == tiles * 16384
     a = lib.moe_forward_workspace_size(0, 64, 2, 8, 4096, 14336, 0)
     b = lib.moe_forward_workspace_size(0, 64, 2, 8, 4096, 14336, 16)
     assert a == b > 0

@@ -60,7 +60,8 @@ def test_align_permute_bit_exact(moe, T, E, k, bm, skew):
     check_permutation(perm, ids.numpy(), E, bm)
 
 
-def expected_packed_bf16(Wg, Wu, Wd):
+def expected_packed_rows(Wg, Wu, Wd):
+    """Packed row order: gate/up rows interleaved by 16, W_d transposed (K-major)."""
     E, H, I = Wg.shape
     gt = Wg.transpose(1, 2).reshape(E, I // 16, 16, H)
     ut = Wu.transpose(1, 2).reshape(E, I // 16, 16, H)
@@ -69,39 +70,48 @@ def expected_packed_bf16(Wg, Wu, Wd):
     return gu.contiguous(), dn
 
 
-@pytest.mark.parametrize("E,H,I", [(3, 128, 192), (2, 256, 64)])
+def tile_image(M, bk):
+    """[E, R, K] -> bytes of 16 KB tiles (128 rows x 128 B), zero-padded, each
+    in the 128-byte-swizzle layout: 16-byte chunk c of row r at c ^ (r % 8)."""
+    E, R, K = M.shape
+    MT, KB = -(-R // 128), -(-K // bk)
+    pad = torch.zeros((E, MT * 128, KB * bk), dtype=M.dtype)
+    pad[:, :R, :K] = M
+    t = pad.view(E, MT, 128, KB, bk).permute(0, 1, 3, 2, 4).contiguous()
+    b = t.view(torch.uint8).view(E, MT, KB, 128, 8, 16)
+    r = torch.arange(128).view(128, 1)
+    c = torch.arange(8).view(1, 8)
+    idx = (c ^ (r % 8)).view(1, 1, 1, 128, 8, 1).expand_as(b)
+    return torch.gather(b, 4, idx).reshape(-1)
+
+
+@pytest.mark.parametrize("E,H,I", [(3, 128, 192), (2, 320, 64)])
 def test_pack_weights_layout(moe, E, H, I):
     L = make_layer("decode", T=1, E=E, H=H, I=I, k=1)
     Wg, Wu, Wd = (W.to(DEV) for W in (L.Wg, L.Wu, L.Wd))
     packed, _ = moe.pack_weights(moe.BF16, Wg, Wu, Wd)
     torch.cuda.synchronize()
-    gu, dn = expected_packed_bf16(L.Wg, L.Wu, L.Wd)
-    p = to_host(packed).view(torch.bfloat16)
-    n = E * 2 * I * H
-    assert torch.equal(p[:n].view(E, 2 * I, H), gu)
-    assert torch.equal(p[n:].view(E, H, I), dn)
+    gu, dn = expected_packed_rows(L.Wg, L.Wu, L.Wd)
+    ref = torch.cat([tile_image(gu, 64), tile_image(dn, 64)])
+    assert torch.equal(to_host(packed), ref)
 
 
 def test_pack_weights_fp8_codes(moe):
-    L = make_layer("fp8", T=1, E=3, H=128, I=192, k=1)
+    E, H, I = 3, 320, 192                       # ragged tiles in both directions
+    L = make_layer("fp8", T=1, E=E, H=H, I=I, k=1)
     Wg, Wu, Wd = (W.to(DEV) for W in (L.Wg, L.Wu, L.Wd))
     packed, scales = moe.pack_weights(moe.FP8_E4M3, Wg, Wu, Wd)
     torch.cuda.synchronize()
-    E, H, I = 3, 128, 192
     codes = {}
     for m, W in enumerate((L.Wg, L.Wu, L.Wd)):
         for e in range(E):
             s, q = oracle.fp8_quantize(W[e])
             assert to_host(scales)[e, m].item() == s
             codes[(m, e)] = torch.from_numpy(q)
-    qg = torch.stack([codes[(0, e)] for e in range(E)])
-    qu = torch.stack([codes[(1, e)] for e in range(E)])
-    qd = torch.stack([codes[(2, e)] for e in range(E)])
-    gu, dn = expected_packed_bf16(qg, qu, qd)
-    p = to_host(packed)
-    n = E * 2 * I * H
-    assert torch.equal(p[:n].view(E, 2 * I, H), gu)
-    assert torch.equal(p[n:].view(E, H, I), dn)
+    qg, qu, qd = (torch.stack([codes[(m, e)] for e in range(E)]) for m in range(3))
+    gu, dn = expected_packed_rows(qg, qu, qd)
+    ref = torch.cat([tile_image(gu, 128), tile_image(dn, 128)])
+    assert torch.equal(to_host(packed), ref)
 
 
 def run_forward(moe, dtype, L, block_m=0, max_ctas=0, ws=None):
