@@ -35,10 +35,10 @@ import torch  # noqa: E402
 from workloads import CONFIGS, make_batch, make_weights  # noqa: E402
 
 WORKLOADS = {
-    "decode": dict(cfg="decode", dtype=0),
-    "prefill": dict(cfg="prefill", dtype=0),
-    "fp8": dict(cfg="fp8", dtype=1),
-    "skewed": dict(cfg="skewed", dtype=0),
+    "decode": dict(cfg="decode", dtype=0, bound="hbm"),
+    "prefill": dict(cfg="prefill", dtype=0, bound="tensor"),
+    "fp8": dict(cfg="fp8", dtype=1, bound="tensor"),      # roofline entry at T=2048
+    "skewed": dict(cfg="skewed", dtype=0, bound="tensor"),
 }
 NBATCH = 4
 # DRAM bytes (read + write) of one gate/up launch from an ncu capture of the
@@ -323,23 +323,37 @@ def run_native(args):
     gu_bytes = {T: statistics.mean(gate_up_bytes(T, k, H, I, a, fp8) for a in active[T])
                 for T in Ts}
     hbm, tf, src = peaks()
+    tpeak = tf * (2 if fp8 else 1)   # e4m3 dense peak = 2x the measured bf16 peak (nominal ratio)
     # dominant kernel: the gate/up GEMM; its largest launch (the largest T)
     Tr = max(Ts)
-    achieved = gu_bytes[Tr] / (gu_ms[Tr] / 1e3) / 1e9
-    agg = sum(gu_bytes[T] for T in Ts) / (sum(gu_ms[T] for T in Ts) / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": TRAFFIC.get((args.workload, Tr)),
-                "kernel": ("grouped_gemm_kernel<%s, gate/up> at T=%d" %
-                           ("e4m3" if fp8 else "bf16", Tr)),
-                "bytes_per_launch": int(gu_bytes[Tr]),
-                "all_T_achieved": round(agg, 1), "all_T_frac": round(agg / hbm, 4),
-                "peak_source": src}
+    gu_flops = {T: 4.0 * T * k * H * I for T in Ts}      # 2 GEMMs of 2*H*I per assignment
+    kname = "grouped_gemm_kernel<%s, gate/up> at T=%d" % ("e4m3" if fp8 else "bf16", Tr)
+    if WORKLOADS[args.workload]["bound"] == "hbm":
+        achieved = gu_bytes[Tr] / (gu_ms[Tr] / 1e3) / 1e9
+        agg = sum(gu_bytes[T] for T in Ts) / (sum(gu_ms[T] for T in Ts) / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4),
+                    "traffic": TRAFFIC.get((args.workload, Tr)), "kernel": kname,
+                    "bytes_per_launch": int(gu_bytes[Tr]),
+                    "all_T_achieved": round(agg, 1), "all_T_frac": round(agg / hbm, 4),
+                    "peak_source": src}
+    else:
+        achieved = gu_flops[Tr] / (gu_ms[Tr] / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak,
+                    "unit": "TFLOP/s", "frac": round(achieved / tpeak, 4),
+                    "traffic": TRAFFIC.get((args.workload, Tr)), "kernel": kname,
+                    "flops_per_launch": int(gu_flops[Tr]),
+                    "peak_source": src + (" (bf16 burst x2 for e4m3)" if fp8 else " (bf16 burst)")}
     wb = 1 if fp8 else 2
     per_T = {}
     for T in Ts:
         a = statistics.mean(active[T])
         layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
+        layer_flops = 6.0 * T * k * H * I
         per_T[str(T)] = {"layer_us": round(1e3 * layer_pdl_ms[T], 2),
+                         "layer_tflops": round(layer_flops / (layer_pdl_ms[T] / 1e3) / 1e12, 1),
+                         "layer_tensor_frac": round(layer_flops / (layer_pdl_ms[T] / 1e3) / 1e12
+                                                    / tpeak, 4),
                          "layer_us_staged": round(1e3 * layer_ms[T], 2),
                          "gate_up_us": round(1e3 * gu_ms[T], 2),
                          "down_us": round(1e3 * dn_ms[T], 2),

@@ -209,7 +209,9 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
 }
 
 // ------------------------------------------------------------------ misc
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+// SiLU(z) = z / (1 + e^-z) with the fast exponential and division intrinsics
+// (relative error ~1e-6, far below the bf16 rounding of h).
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // Ordered-int encoding of a non-negative float for atomicMax.
 __device__ __forceinline__ void atomic_max_nonneg(uint32_t* addr, float v) {

@@ -13,16 +13,20 @@ constexpr int kThreads = 256;
 constexpr int kRowsPerBlock = kThreads / 32;
 
 // a3: X_perm[p] = x[sorted_ids[p] / k] for p < offsets[E]; pad rows are zero.
+// Also w_perm[p] = w[sorted_ids[p]] (0 for pads), the routing weight the down
+// GEMM's epilogue applies to row p.
 __global__ void __launch_bounds__(kThreads)
     gather_bf16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
                        const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
-                       int capacity, uint4* __restrict__ x_perm) {
+                       int capacity, const float* __restrict__ w, uint4* __restrict__ x_perm,
+                       float* __restrict__ w_perm) {
     pdl_wait();
     pdl_trigger();
     const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (p >= capacity || p >= offsets[E]) return;
     const int sid = sorted_ids[p];
+    if (lane == 0) w_perm[p] = sid >= 0 ? w[sid] : 0.0f;
     uint4* dst = x_perm + static_cast<long>(p) * vec_per_row;
     if (sid < 0) {
         for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
@@ -80,13 +84,15 @@ __global__ void __launch_bounds__(kThreads)
     gather_fp8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
                       const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
                       int capacity, const uint32_t* __restrict__ amax_bits,
-                      uint2* __restrict__ x_perm) {
+                      const float* __restrict__ w, uint2* __restrict__ x_perm,
+                      float* __restrict__ w_perm) {
     pdl_wait();
     pdl_trigger();
     const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (p >= capacity || p >= offsets[E]) return;
     const int sid = sorted_ids[p];
+    if (lane == 0) w_perm[p] = sid >= 0 ? w[sid] : 0.0f;
     uint2* dst = x_perm + static_cast<long>(p) * vec_per_row;
     if (sid < 0) {
         for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint2(0, 0);
@@ -244,11 +250,12 @@ int blocks_for(long n, int per_block, int cap) {
 }  // namespace
 
 cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                               int E, int k, int H, int capacity, void* x_perm, cudaStream_t s) {
+                               int E, int k, int H, int capacity, const float* w, void* x_perm,
+                               float* w_perm, cudaStream_t s) {
     if (capacity == 0) return cudaSuccess;
     return launch_pdl(gather_bf16_kernel, dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock),
                       dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
-                      k, H / 8, capacity, static_cast<uint4*>(x_perm));
+                      k, H / 8, capacity, w, static_cast<uint4*>(x_perm), w_perm);
 }
 
 cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s) {
@@ -259,11 +266,11 @@ cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaS
 
 cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
                               int E, int k, int H, int capacity, const uint32_t* amax_bits,
-                              void* x_perm, cudaStream_t s) {
+                              const float* w, void* x_perm, float* w_perm, cudaStream_t s) {
     if (capacity == 0) return cudaSuccess;
     return launch_pdl(gather_fp8_kernel, dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock),
                       dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
-                      k, H / 8, capacity, amax_bits, static_cast<uint2*>(x_perm));
+                      k, H / 8, capacity, amax_bits, w, static_cast<uint2*>(x_perm), w_perm);
 }
 
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,

@@ -13,23 +13,26 @@
 // Work decomposition ("dynamic scheduling of variable token groups", "FP8
 // esetén a Triton backend bizonyult gyorsabbnak"): for every expert e with
 // c_e tokens, units = ceil(Mw/128) weight tiles x ceil(c_e/nmax) token tiles,
-// each with KB = ceil(K/BK) k-blocks of 128 bytes.  All units' k-blocks form
-// one linear space that is cut into equal contiguous ranges, one per CTA
-// (stream-K).  Units that straddle a range boundary are finished by whichever
-// contributor arrives last, which sums the fp32 partials in CTA order -- a
-// fixed order, so the result does not depend on timing.
+// each with KB = ceil(K/BK) k-blocks of 128 bytes.  Units are ordered by cost
+// (full token tiles first, then partial ones, largest first) and dealt
+// round-robin in waves to the persistent CTAs; the last one to two waves are
+// cut into equal contiguous k-block ranges instead (stream-K), so all CTAs
+// finish together.  Units that straddle a range boundary are finished by
+// whichever contributor arrives last, which sums the fp32 partials in CTA
+// order -- a fixed order, so the result does not depend on timing.
 //
-// Roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer (single
-// thread), warp 2 = TMEM allocator, warps 4-7 = epilogue (TMEM lanes 0-127).
-// smem ring of `stages` (A 16 KB + B nmax*128 B), 128-byte swizzle; two TMEM
+// Roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (single
+// thread), warp 2 = TMEM allocator, warps 4-11 = epilogue (two warps per
+// 32-lane TMEM quarter, alternating 16-column chunks).
+// smem ring of 2 stages of kps k-blocks (A kps*16 KB + B kps*nmax*128 B),
+// 128-byte swizzle; two TMEM
 // accumulators of nmax fp32 columns so the epilogue of one unit overlaps the
 // main loop of the next.  Every wait is bounded; on expiry the kernel records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 //
 // Weights (A) are pre-packed as 16 KB tiles that are already the swizzled
-// shared-memory image of one stage, so each stage's A operand is one
-// contiguous bulk copy and a CTA's stream-K range is one sequential stream
-// through memory.  Activations (B) come through TMA tensor maps with 64-row
+// shared-memory image of one stage, so a stage's A operand (one to four
+// consecutive k-blocks) is one contiguous bulk copy.  Activations (B) come through TMA tensor maps with 64-row
 // and 16-row boxes, so a token tile moves only its own rows.  Launched with
 // programmatic dependent launch: the producer fetches the first weight tiles
 // before waiting for the previous kernel, whose output (B) it loads after.
@@ -45,11 +48,12 @@ namespace {
 constexpr int kBM = 128;            // weight rows per tile (UMMA M)
 constexpr int kRowBytes = 128;      // K bytes per stage row (one swizzle atom)
 constexpr int kATileBytes = kBM * kRowBytes;
-constexpr int kThreads = 256;
-constexpr int kEpiWarp0 = 4;
+constexpr int kThreads = 384;
+constexpr int kEpiWarp0 = 4;          // warps 4..11: two per TMEM lane quarter
+constexpr int kEpiThreads = 256;
 constexpr int kMaxStages = 12;
 constexpr int kMinKbPerCta = 4;
-constexpr int kStagingBytes = 4 * 1024;
+constexpr int kStagingBytes = 8 * 1024;
 constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
 constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
@@ -61,8 +65,7 @@ struct GemmArgs {
     void* out;
     const int32_t* counts;
     const int32_t* offsets;
-    const float* route_w;
-    const int32_t* sorted_ids;
+    const float* w_perm;       // routing weight of each permuted row (0 for pads)
     const float* w_scales;
     const uint32_t* act_amax;
     uint32_t* out_amax;
@@ -83,10 +86,14 @@ struct Ctl {
     uint32_t prod_pos;   // k-blocks issued by the producer
     uint32_t mma_pos;    // k-blocks whose full barrier the MMA thread observed
     uint32_t mma_issued; // 1 once any MMA was issued
-    int scan_tmp[9];
-    int unit_prefix[kMaxExperts + 1];
-    int ntt[kMaxExperts];
-    int cnt[kMaxExperts];
+    int scan_tmp[kThreads / 32 + 1];
+    int n_full_units;                  // units of full token tiles (N = nmax)
+    int n_partial;                     // experts with a partial last token tile
+    int full_prefix[kMaxExperts + 1];  // full-tile units before expert e
+    int nfull[kMaxExperts];            // full token tiles of expert e
+    int np[kMaxExperts];               // rows of e's partial tile (0: none)
+    int key[kMaxExperts];              // sort key of the partial tiles
+    int part_expert[kMaxExperts];      // experts with a partial tile, largest first
     int off[kMaxExperts];
 };
 
@@ -106,24 +113,73 @@ __device__ __forceinline__ int find_expert(const int* prefix, int E, int u) {
     return lo;
 }
 
-__device__ __forceinline__ Seg make_seg(const Ctl& c, const GemmArgs& g, long long x,
-                                        long long we) {
+// Unit order (cost first): all units of full token tiles (N = nmax) in
+// (expert, weight tile, token tile) order, then the units of every expert's
+// partial last token tile, largest first, in (expert, weight tile) order.
+// Dealt round-robin, each wave then holds units of similar cost, and the
+// stream-K remainder is made of the cheapest ones.
+__device__ __forceinline__ Seg make_seg(const Ctl& c, const GemmArgs& g, int u, int kb0, int kb1) {
     Seg s;
-    s.u = static_cast<int>(x / g.KB);
-    s.kb0 = static_cast<int>(x - static_cast<long long>(s.u) * g.KB);
-    const long long left = we - x;
-    s.kb1 = (g.KB - s.kb0 <= left) ? g.KB : s.kb0 + static_cast<int>(left);
-    s.e = find_expert(c.unit_prefix, g.E, s.u);
-    const int local = s.u - c.unit_prefix[s.e];
-    const int ntt = c.ntt[s.e];
-    s.m = local / ntt;
-    const int nt = local - s.m * ntt;
+    s.u = u;
+    s.kb0 = kb0;
+    s.kb1 = kb1;
+    int nt;
+    if (u < c.n_full_units) {
+        s.e = find_expert(c.full_prefix, g.E, u);
+        const int local = u - c.full_prefix[s.e];
+        const int nf = c.nfull[s.e];
+        s.m = local / nf;
+        nt = local - s.m * nf;
+        s.N = g.nmax;
+    } else {
+        const int v = u - c.n_full_units;
+        const int r = v / g.MT;
+        s.m = v - r * g.MT;
+        s.e = c.part_expert[r];
+        nt = c.nfull[s.e];
+        s.N = c.np[s.e];
+    }
     s.b_row = c.off[s.e] + nt * g.nmax;
-    const int rem = c.cnt[s.e] - nt * g.nmax;
-    const int n = rem < g.nmax ? rem : g.nmax;
-    s.N = (n + 15) & ~15;
     return s;
 }
+
+// Work of one CTA.  With U units and G CTAs: when U > G, all but the last
+// full wave are dealt whole and round-robin (CTA c takes units c, c+G, ...;
+// each wave works on adjacent units, which share weight and token tiles in
+// L2 and stream adjacent weight memory); the remaining G..2G-1 units are cut
+// stream-K style into equal contiguous k-block ranges, one per CTA, so every
+// CTA ends at the same time.  When U <= G, everything is stream-K.
+struct Sched {
+    int n_dp;          // whole units dealt round-robin
+    int unit0;         // first unit of the stream-K part
+    long long L;       // k-blocks of the stream-K part
+    int Gsk;           // CTAs sharing the stream-K part
+    long long ws, we;  // this CTA's stream-K range
+};
+
+struct Cursor {
+    int j, n_dp, cta, G, KB, unit0;
+    long long x, we;
+    __device__ __forceinline__ bool next(int& u, int& kb0, int& kb1) {
+        if (j < n_dp) {
+            u = cta + j * G;
+            kb0 = 0;
+            kb1 = KB;
+            ++j;
+            return true;
+        }
+        if (x < we) {
+            const long long uu = x / KB;
+            u = unit0 + static_cast<int>(uu);
+            kb0 = static_cast<int>(x - uu * KB);
+            const long long left = we - x;
+            kb1 = (KB - kb0 <= left) ? KB : kb0 + static_cast<int>(left);
+            x += kb1 - kb0;
+            return true;
+        }
+        return false;
+    }
+};
 
 // CTA whose range [floor(c*L/G), floor((c+1)*L/G)) holds k-block X.
 __device__ __forceinline__ int owner_cta(long long X, long long L, int G) {
@@ -131,7 +187,7 @@ __device__ __forceinline__ int owner_cta(long long X, long long L, int G) {
 }
 
 __device__ __forceinline__ void named_bar_epi() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 __device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
@@ -139,19 +195,25 @@ __device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
     *reinterpret_cast<volatile int*>(&c.abort) = 1;
 }
 
+// One 16-column chunk (16 tokens) of the accumulator rows this thread owns.
+// Epilogue warp w (4..11) owns TMEM lane quarter q = w % 4 (rows 32q..32q+31)
+// and every other chunk (half h = (w - 4) / 4).  `sw` is the FP8 dequant
+// factor of this row; `wreg` holds the routing weights of the unit's tokens,
+// token t in lane t/8, register t%8.
 template <bool FP8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int c0, float (&v)[16],
-                                               float act_scale, uint8_t* staging, float& amax) {
-    const int wq = (threadIdx.x >> 5) - kEpiWarp0;
+                                               float sw, const float (&wreg)[8], uint8_t* staging,
+                                               float& amax) {
+    const int ew = (threadIdx.x >> 5) - kEpiWarp0;
+    const int q = (threadIdx.x >> 5) & 3;
     const int lane = threadIdx.x & 31;
     constexpr unsigned kFull = 0xffffffffu;
-    if constexpr (EPI == 0) {
-        if constexpr (FP8) {
-            const float sw = g.w_scales[s.e * 3 + (lane < 16 ? 0 : 1)] * act_scale;
+    if constexpr (FP8) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= sw;
-        }
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + wq * 1024);
+        for (int i = 0; i < 16; ++i) v[i] *= sw;
+    }
+    if constexpr (EPI == 0) {
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + ew * 1024);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float p = __shfl_xor_sync(kFull, v[i], 16);
@@ -165,30 +227,20 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
         }
         __syncwarp();
         const int row = s.b_row + c0 + (lane >> 1);
-        const int col = s.m * 64 + 16 * wq + 8 * (lane & 1);
+        const int col = s.m * 64 + 16 * q + 8 * (lane & 1);
         const uint4 val = *reinterpret_cast<const uint4*>(st + (lane >> 1) * 16 + 8 * (lane & 1));
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
                                   static_cast<long>(row) * g.ldo + col) = val;
         __syncwarp();
     } else {
-        if constexpr (FP8) {
-            const float sw = g.w_scales[s.e * 3 + 2] * act_scale;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= sw;
-        }
-        float wt = 0.0f;
-        if (lane < 16) {
-            const int sid = __ldcg(g.sorted_ids + s.b_row + c0 + lane);
-            wt = sid >= 0 ? __ldcg(g.route_w + sid) : 0.0f;
-        }
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + wq * 1024);
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + ew * 1024);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const float wi = __shfl_sync(kFull, wt, i);
+            const float wi = __shfl_sync(kFull, wreg[i & 7], (c0 + i) >> 3);
             st[i * 32 + lane] = __float2bfloat16_rn(v[i] * wi);
         }
         __syncwarp();
-        const int hcol0 = s.m * kBM + 32 * wq;
+        const int hcol0 = s.m * kBM + 32 * q;
         if (hcol0 < g.Mvalid) {
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -227,14 +279,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
         const int e = threadIdx.x;
         int units = 0;
+        int key = 0x7fffffff;
         if (e < g.E) {
             const int c = __ldcg(g.counts + e);
-            ctl.cnt[e] = c;
             ctl.off[e] = __ldcg(g.offsets + e);
-            const int nt = (c + g.nmax - 1) / g.nmax;
-            ctl.ntt[e] = nt;
-            units = nt * g.MT;
+            int nf = c / g.nmax;
+            const int r = c - nf * g.nmax;
+            int n = (r + 15) & ~15;
+            if (n == g.nmax) {  // rounds up to a full tile
+                ++nf;
+                n = 0;
+            }
+            ctl.nfull[e] = nf;
+            ctl.np[e] = n;
+            units = nf * g.MT;
+            if (n > 0) key = (g.nmax - n) * kMaxExperts + e;
         }
+        if (e < kMaxExperts) ctl.key[e] = key;
         int inc = units;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -249,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&ctl.tfull[i], 1);
-                mbar_init(&ctl.tempty[i], 128);
+                mbar_init(&ctl.tempty[i], kEpiThreads);
             }
             mbar_init(&ctl.drain, 1);
             fence_mbar_init();
@@ -274,24 +335,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ctl.scan_tmp[i] = run;
                 run += t;
             }
-            ctl.scan_tmp[8] = run;
+            ctl.scan_tmp[kThreads / 32] = run;
         }
         __syncthreads();
-        if (e < g.E) ctl.unit_prefix[e] = ctl.scan_tmp[warp] + inc - units;
-        if (threadIdx.x == 0) ctl.unit_prefix[g.E] = ctl.scan_tmp[8];
+        if (e < g.E) ctl.full_prefix[e] = ctl.scan_tmp[warp] + inc - units;
+        if (threadIdx.x == 0) {
+            ctl.full_prefix[g.E] = ctl.scan_tmp[kThreads / 32];
+            ctl.n_full_units = ctl.scan_tmp[kThreads / 32];
+        }
+        // rank of e's partial tile among all partial tiles (keys are distinct)
+        if (key != 0x7fffffff) {
+            int rank = 0;
+            for (int i = 0; i < g.E; ++i) rank += ctl.key[i] < key ? 1 : 0;
+            ctl.part_expert[rank] = e;
+        }
+        const int n_has = __popc(__ballot_sync(0xffffffffu, key != 0x7fffffff));
+        __syncthreads();
+        if (lane == 0) ctl.scan_tmp[warp] = n_has;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+            for (int i = 0; i < kThreads / 32; ++i) t += ctl.scan_tmp[i];
+            ctl.n_partial = t;
+        }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
 
-    const long long L = static_cast<long long>(ctl.unit_prefix[g.E]) * g.KB;
-    long long G = (L + kMinKbPerCta - 1) / kMinKbPerCta;
-    if (G > gridDim.x) G = gridDim.x;
-    if (G < 1) G = 1;
+    const int U = ctl.n_full_units + ctl.n_partial * g.MT;
+    const int G = gridDim.x;
     const int cta = blockIdx.x;
-    const bool active = L > 0 && cta < G;
-    const long long ws = active ? static_cast<long long>(cta) * L / G : 0;
-    const long long we = active ? static_cast<long long>(cta + 1) * L / G : 0;
+    Sched sc;
+    sc.n_dp = U > G ? U / G - 1 : 0;
+    sc.unit0 = sc.n_dp * G;
+    sc.L = static_cast<long long>(U - sc.unit0) * g.KB;
+    {
+        long long gs = (sc.L + kMinKbPerCta - 1) / kMinKbPerCta;
+        sc.Gsk = static_cast<int>(gs < G ? gs : G);
+        if (sc.Gsk < 1) sc.Gsk = 1;
+    }
+    const bool in_sk = sc.L > 0 && cta < sc.Gsk;
+    sc.ws = in_sk ? static_cast<long long>(cta) * sc.L / sc.Gsk : 0;
+    sc.we = in_sk ? static_cast<long long>(cta + 1) * sc.L / sc.Gsk : 0;
+    const bool active = sc.n_dp > 0 || in_sk;
+    auto cursor = [&]() { return Cursor{0, sc.n_dp, cta, G, g.KB, sc.unit0, sc.ws, sc.we}; };
     const uint32_t tmem_base = ctl.tmem_base;
     const int S = g.stages;
 
@@ -304,8 +392,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // previous kernel; their activation rows follow after it.
             int early = 0;
             if (active) {
-                for (long long x = ws; x < we && early < S;) {
-                    const Seg s = make_seg(ctl, g, x, we);
+                Cursor cur = cursor();
+                int u, kb0, kb1;
+                while (early < S && cur.next(u, kb0, kb1)) {
+                    const Seg s = make_seg(ctl, g, u, kb0, kb1);
                     const uint8_t* a = g.a_tiles +
                                        (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
                     const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
@@ -317,13 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   a + static_cast<size_t>(kb) * kTileBytes, nk * kATileBytes,
                                   &ctl.full[early], kEvictFirst);
                     }
-                    x += s.kb1 - s.kb0;
                 }
             }
             pdl_wait();
             pdl_trigger();
-            for (long long x = ws; active && x < we;) {
-                const Seg s = make_seg(ctl, g, x, we);
+            Cursor cur = cursor();
+            int u, kb0, kb1;
+            while (active && cur.next(u, kb0, kb1)) {
+                const Seg s = make_seg(ctl, g, u, kb0, kb1);
                 const uint8_t* a = g.a_tiles +
                                    (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
                 const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
@@ -355,7 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (!ok) break;
-                x += s.kb1 - s.kb0;
             }
             ctl.prod_pos = it > static_cast<uint32_t>(early) ? it : static_cast<uint32_t>(early);
         }
@@ -365,8 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && active) {
             uint32_t it = 0, si = 0;
             bool ok = true;
-            for (long long x = ws; x < we && ok; ++si) {
-                const Seg s = make_seg(ctl, g, x, we);
+            Cursor cur = cursor();
+            int u, kb0, kb1;
+            for (; ok && cur.next(u, kb0, kb1); ++si) {
+                const Seg s = make_seg(ctl, g, u, kb0, kb1);
                 const int acc = si & 1;
                 if (!mbar_wait(&ctl.tempty[acc], ((si >> 1) & 1u) ^ 1u, &ctl.abort)) {
                     raise_abort(ctl, g.status);
@@ -399,50 +491,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 umma_commit(&ctl.tfull[acc]);
-                x += s.kb1 - s.kb0;
             }
             ctl.mma_pos = it;
         }
         __syncwarp();
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------ epilogue
-        const int wq = warp - kEpiWarp0;
-        const int row = 32 * wq + lane;  // accumulator row = TMEM lane
+        const int q = warp & 3;                     // TMEM lane quarter
+        const int half = (warp - kEpiWarp0) >> 2;   // which chunks: c0 = 16*(2j + half)
+        const int row = 32 * q + lane;              // accumulator row = TMEM lane
         float act_scale = 1.0f;
         if constexpr (FP8) act_scale = fp8_scale_from_amax(__ldcg(g.act_amax));
         float amax = 0.0f;
         uint32_t si = 0;
-        for (long long x = ws; active && x < we; ++si) {
-            const Seg s = make_seg(ctl, g, x, we);
+        Cursor cur = cursor();
+        int u, kb0, kb1;
+        for (; active && cur.next(u, kb0, kb1); ++si) {
+            const Seg s = make_seg(ctl, g, u, kb0, kb1);
             const int acc = si & 1;
+            // per-unit constants: FP8 dequant factor of this row, routing weights
+            float sw = 1.0f;
+            if constexpr (FP8)
+                sw = act_scale * __ldg(g.w_scales + s.e * 3 + (EPI == 1 ? 2 : (lane < 16 ? 0 : 1)));
+            float wreg[8];
+            if constexpr (EPI == 1) {
+                if (8 * lane < s.N) {
+                    const float4* wp = reinterpret_cast<const float4*>(g.w_perm + s.b_row + 8 * lane);
+                    const float4 a = __ldcg(wp), b = __ldcg(wp + 1);
+                    wreg[0] = a.x; wreg[1] = a.y; wreg[2] = a.z; wreg[3] = a.w;
+                    wreg[4] = b.x; wreg[5] = b.y; wreg[6] = b.z; wreg[7] = b.w;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) wreg[i] = 0.0f;
+                }
+            }
             if (!mbar_wait(&ctl.tfull[acc], (si >> 1) & 1u, &ctl.abort)) {
                 raise_abort(ctl, g.status);
                 break;
             }
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + acc * g.nmax;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * g.nmax;
             if (s.kb0 == 0 && s.kb1 == g.KB) {
-                for (int c0 = 0; c0 < s.N; c0 += 16) {
+                for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
                     tmem_ld16(taddr + c0, v);
-                    epilogue_chunk<FP8, EPI>(g, s, c0, v, act_scale, staging, amax);
+                    epilogue_chunk<FP8, EPI>(g, s, c0, v, sw, wreg, staging, amax);
                 }
                 tc_fence_before();
                 mbar_arrive(&ctl.tempty[acc]);
             } else {
-                const long long X0 = static_cast<long long>(s.u) * g.KB;
-                const int cf = owner_cta(X0, L, static_cast<int>(G));
-                const int cl = owner_cta(X0 + g.KB - 1, L, static_cast<int>(G));
+                const long long X0 = static_cast<long long>(s.u - sc.unit0) * g.KB;
+                const int cf = owner_cta(X0, sc.L, sc.Gsk);
+                const int cl = owner_cta(X0 + g.KB - 1, sc.L, sc.Gsk);
                 const long long slot_elems = static_cast<long long>(kBM) * g.nmax;
                 float* mine = g.partials + (2LL * cta + (cta == cf ? 1 : 0)) * slot_elems +
                               static_cast<long long>(row) * g.nmax;
-                for (int c0 = 0; c0 < s.N; c0 += 16) {
+                for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
                     tmem_ld16(taddr + c0, v);
                     float4* p4 = reinterpret_cast<float4*>(mine + c0);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        p4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    for (int i = 0; i < 4; ++i)
+                        p4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
                 tc_fence_before();
                 mbar_arrive(&ctl.tempty[acc]);
@@ -457,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 named_bar_epi();
                 if (finisher) {
                     __threadfence();
-                    for (int c0 = 0; c0 < s.N; c0 += 16) {
+                    for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                         float v[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) v[i] = 0.0f;
@@ -468,12 +578,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i);
                         }
-                        epilogue_chunk<FP8, EPI>(g, s, c0, v, act_scale, staging, amax);
+                        epilogue_chunk<FP8, EPI>(g, s, c0, v, sw, wreg, staging, amax);
                     }
                     if (threadIdx.x == kEpiWarp0 * 32) g.counters[cf] = 0;
                 }
             }
-            x += s.kb1 - s.kb0;
         }
         if constexpr (FP8 && EPI == 0) {
 #pragma unroll
@@ -572,7 +681,8 @@ int gemm_nmax_for(int T, int k, int E) {
     const long mean2 = (2L * T * k + E - 1) / E;
     long n = (mean2 + 15) & ~15L;
     if (n < 16) n = 16;
-    return static_cast<int>(n > 256 ? 256 : n);
+    if (n > 256) n = 256;
+    return static_cast<int>(n);
 }
 
 size_t gemm_partials_bytes(int nmax) {
@@ -589,12 +699,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.KB = p.KB;
     g.MT = p.MT;
     g.a_tiles = static_cast<const uint8_t*>(p.weights);
-    // Weight streaming (small token tiles): 4 k-blocks per stage, i.e. 64 KB
-    // bulk copies, two stages (~128 KB in flight per SM) -- measured on B200
-    // to sustain a higher HBM read rate than more, smaller copies.  Large
-    // token tiles are tensor-bound and keep one k-block per stage.
-    const int kps = p.nmax <= 64 ? 4 : 1;
-    const int max_stages = p.nmax <= 64 ? 2 : kMaxStages;
+    // Two stages of several k-blocks each: small token tiles (weight
+    // streaming) take 4 k-blocks (64 KB weight copies), large ones 2 (32 KB
+    // weights + 64 KB activations).  Measured on B200: fewer, larger copies
+    // sustain more bandwidth than many 16 KB stages, for both regimes.
+    const int kps = p.nmax <= 64 ? 4 : 2;
+    const int max_stages = 2;
     const int stage_bytes = kps * (kATileBytes + p.nmax * kRowBytes);
     int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
     if (stages > max_stages) stages = max_stages;
@@ -606,8 +716,7 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.out = p.out;
     g.counts = p.counts;
     g.offsets = p.offsets;
-    g.route_w = p.route_w;
-    g.sorted_ids = p.sorted_ids;
+    g.w_perm = p.w_perm;
     g.w_scales = p.w_scales;
     g.act_amax = p.act_amax;
     g.out_amax = p.out_amax;

@@ -75,12 +75,14 @@ cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int bl
                                  cudaStream_t s);
 
 // ---- a3/a5/a7 and packing (elementwise.cu)
+// The gathers also write w_perm[p] = w[sorted_ids[p]] (0 for pads).
 cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                               int E, int k, int H, int capacity, void* x_perm, cudaStream_t s);
+                               int E, int k, int H, int capacity, const float* w, void* x_perm,
+                               float* w_perm, cudaStream_t s);
 cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s);
 cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
                               int E, int k, int H, int capacity, const uint32_t* amax_bits,
-                              void* x_perm, cudaStream_t s);
+                              const float* w, void* x_perm, float* w_perm, cudaStream_t s);
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
                                   int capacity, const uint32_t* amax_bits, void* h_q,
                                   cudaStream_t s);
@@ -106,8 +108,7 @@ struct GemmProblem {
     int ldo;
     const int32_t* counts;
     const int32_t* offsets;
-    const float* route_w;        // epi 1
-    const int32_t* sorted_ids;   // epi 1
+    const float* w_perm;         // epi 1: routing weight per permuted row
     const float* w_scales;       // [E][3] (FP8)
     const uint32_t* act_amax;    // FP8: amax bits of the activation operand
     uint32_t* out_amax;          // FP8 epi 0: amax of h (bits)

@@ -58,6 +58,7 @@ struct Carver {
 
 struct FfnBuffers {
     int32_t* ctl;
+    float* w_perm;
     void* x_perm;
     void* h;
     void* h_q;
@@ -66,6 +67,7 @@ struct FfnBuffers {
 
 void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int cap, int H, int I, int nmax) {
     const size_t elt = dt == MOE_FP8_E4M3 ? 1 : 2;
+    b.w_perm = c.take<float>(sizeof(float) * static_cast<size_t>(cap > 0 ? cap : 1));
     b.x_perm = c.take<void>(static_cast<size_t>(cap) * H * elt);
     b.h = c.take<void>(static_cast<size_t>(cap) * I * 2);
     b.h_q = dt == MOE_FP8_E4M3 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
@@ -111,9 +113,10 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
         e = launch_amax_bf16(f.x, static_cast<long>(f.T) * f.H, amax_x, s);
         if (e == cudaSuccess)
             e = launch_gather_fp8(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, amax_x,
-                                  b.x_perm, s);
+                                  f.w, b.x_perm, b.w_perm, s);
     } else {
-        e = launch_gather_bf16(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, b.x_perm, s);
+        e = launch_gather_bf16(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, f.w, b.x_perm,
+                               b.w_perm, s);
     }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 2, s);
@@ -162,8 +165,7 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     dn.act = fp8 ? b.h_q : b.h;
     dn.out = f.y_perm;
     dn.ldo = f.H;
-    dn.route_w = f.w;
-    dn.sorted_ids = f.sorted_ids;
+    dn.w_perm = b.w_perm;
     dn.act_amax = amax_h;
     dn.out_amax = nullptr;
     dn.counters = b.ctl + kCtlCountersDn;
