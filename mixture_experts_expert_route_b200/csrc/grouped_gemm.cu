@@ -36,6 +36,7 @@
 // and 16-row boxes, so a token tile moves only its own rows.  Launched with
 // programmatic dependent launch: the producer fetches the first weight tiles
 // before waiting for the previous kernel, whose output (B) it loads after.
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -58,7 +59,7 @@ constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
 constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
 struct GemmArgs {
-    int E, Mw, K, KB, MT, Mvalid;
+    int E, Mw, K, KB, MT, MTu, Mvalid;   // MTu: weight tiles per unit step (MT, or pairs)
     int nmax, stages, kps, tmem_cols;
     const uint8_t* a_tiles;
     int ldo;
@@ -98,7 +99,8 @@ struct Ctl {
 };
 
 struct Seg {
-    int u, kb0, kb1, e, m, b_row, N;
+    int u, kb0, kb1, e, m, b_row, N;  // N: valid token rows rounded to 16
+    int Nm;                           // MMA N (a CTA pair needs a multiple of 32)
 };
 
 constexpr int kDynSmemMax = kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024;
@@ -118,6 +120,7 @@ __device__ __forceinline__ int find_expert(const int* prefix, int E, int u) {
 // partial last token tile, largest first, in (expert, weight tile) order.
 // Dealt round-robin, each wave then holds units of similar cost, and the
 // stream-K remainder is made of the cheapest ones.
+template <bool PAIR>
 __device__ __forceinline__ Seg make_seg(const Ctl& c, const GemmArgs& g, int u, int kb0, int kb1) {
     Seg s;
     s.u = u;
@@ -133,13 +136,14 @@ __device__ __forceinline__ Seg make_seg(const Ctl& c, const GemmArgs& g, int u, 
         s.N = g.nmax;
     } else {
         const int v = u - c.n_full_units;
-        const int r = v / g.MT;
-        s.m = v - r * g.MT;
+        const int r = v / g.MTu;
+        s.m = v - r * g.MTu;
         s.e = c.part_expert[r];
         nt = c.nfull[s.e];
         s.N = c.np[s.e];
     }
     s.b_row = c.off[s.e] + nt * g.nmax;
+    s.Nm = PAIR ? ((s.N + 31) & ~31) : s.N;
     return s;
 }
 
@@ -201,9 +205,9 @@ __device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
 // factor of this row; `wreg` holds the routing weights of the unit's tokens,
 // token t in lane t/8, register t%8.
 template <bool FP8, int EPI>
-__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int c0, float (&v)[16],
-                                               float sw, const float (&wreg)[8], uint8_t* staging,
-                                               float& amax) {
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int m_own, int c0,
+                                               float (&v)[16], float sw, const float (&wreg)[8],
+                                               uint8_t* staging, float& amax) {
     const int ew = (threadIdx.x >> 5) - kEpiWarp0;
     const int q = (threadIdx.x >> 5) & 3;
     const int lane = threadIdx.x & 31;
@@ -227,10 +231,11 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
         }
         __syncwarp();
         const int row = s.b_row + c0 + (lane >> 1);
-        const int col = s.m * 64 + 16 * q + 8 * (lane & 1);
+        const int col = m_own * 64 + 16 * q + 8 * (lane & 1);
         const uint4 val = *reinterpret_cast<const uint4*>(st + (lane >> 1) * 16 + 8 * (lane & 1));
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
-                                  static_cast<long>(row) * g.ldo + col) = val;
+        if (m_own < g.MT)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                      static_cast<long>(row) * g.ldo + col) = val;
         __syncwarp();
     } else {
         __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + ew * 1024);
@@ -240,7 +245,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
             st[i * 32 + lane] = __float2bfloat16_rn(v[i] * wi);
         }
         __syncwarp();
-        const int hcol0 = s.m * kBM + 32 * q;
+        const int hcol0 = m_own * kBM + 32 * q;
         if (hcol0 < g.Mvalid) {
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -256,9 +261,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
     }
 }
 
-template <bool FP8, int EPI>
+template <bool FP8, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB64,
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ Ctl ctl;
@@ -268,8 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stage = kps consecutive k-blocks: A kps*16 KB (one bulk copy), B kps
     // slots of nmax rows x 128 B
     const int KPS = g.kps;
+    const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
     const int a_stage_bytes = KPS * kATileBytes;
-    const int b_kb_bytes = g.nmax * kRowBytes;
+    // a pair member holds half of each token tile
+    const int b_kb_bytes = (PAIR ? g.nmax / 2 : g.nmax) * kRowBytes;
     const int b_stage_bytes = KPS * b_kb_bytes;
     uint8_t* smA = base;
     uint8_t* smB = smA + g.stages * a_stage_bytes;
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ctl.nfull[e] = nf;
             ctl.np[e] = n;
-            units = nf * g.MT;
+            units = nf * g.MTu;
             if (n > 0) key = (g.nmax - n) * kMaxExperts + e;
         }
         if (e < kMaxExperts) ctl.key[e] = key;
@@ -310,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&ctl.tfull[i], 1);
-                mbar_init(&ctl.tempty[i], kEpiThreads);
+                mbar_init(&ctl.tempty[i], (PAIR ? 2 : 1) * (kEpiThreads / 32));
             }
             mbar_init(&ctl.drain, 1);
             fence_mbar_init();
@@ -320,12 +328,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl.mma_issued = 0;
         }
         if (warp == 0 && lane == 0) {
+            if constexpr (PAIR) tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB64);
             tma_prefetch_desc(&tmB16);
         }
         if (warp == 2) {
-            tmem_alloc(&ctl.tmem_base, g.tmem_cols);
-            tmem_relinquish();
+            if constexpr (PAIR) {
+                tmem_alloc_pair(&ctl.tmem_base, g.tmem_cols);
+                tmem_relinquish_pair();
+            } else {
+                tmem_alloc(&ctl.tmem_base, g.tmem_cols);
+                tmem_relinquish();
+            }
         }
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -361,11 +375,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        // the peer's barriers must be initialised before any cross-CTA signal
+        if constexpr (PAIR) cluster_sync();
     }
 
-    const int U = ctl.n_full_units + ctl.n_partial * g.MT;
-    const int G = gridDim.x;
-    const int cta = blockIdx.x;
+    const int U = ctl.n_full_units + ctl.n_partial * g.MTu;
+    const int G = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const int cta = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     Sched sc;
     sc.n_dp = U > G ? U / G - 1 : 0;
     sc.unit0 = sc.n_dp * G;
@@ -385,9 +401,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // (both CTAs of a pair run it; their copies complete on the rank-0
+        // CTA's barrier, which the rank-0 producer arms for both)
         if (lane == 0) {
             uint32_t it = 0;
             const int bk_elems = FP8 ? 128 : 64;
+            const int mt_last = g.MT - 1;
+            // A pair loads full KPS-tile boxes of weights; a single CTA loads
+            // exactly the stage's k-blocks.
+            auto stage_bytes = [&](const Seg& sg, int nk) -> uint32_t {
+                const int rows = PAIR ? sg.Nm / 2 : sg.N;
+                const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
+                const uint32_t b = static_cast<uint32_t>(nk * (n64 * 64 + n16 * 16) * kRowBytes);
+                return PAIR ? 2u * (static_cast<uint32_t>(KPS * kATileBytes) + b)
+                            : static_cast<uint32_t>(nk * kATileBytes) + b;
+            };
+            auto load_a = [&](const Seg& sg, int kb, int nk, int st) {
+                int m_own = PAIR ? 2 * sg.m + rank : sg.m;
+                if (m_own > mt_last) m_own = mt_last;   // odd tile count: any valid tile
+                const size_t tile = (static_cast<size_t>(sg.e) * g.MT + m_own) * g.KB + kb;
+                if constexpr (PAIR)
+                    tma_load_2d_pair(smA + st * a_stage_bytes, &tmA, &ctl.full[st], 0,
+                                     static_cast<int>(tile * kTileRows), kEvictFirst);
+                else
+                    bulk_load(smA + st * a_stage_bytes, g.a_tiles + tile * kTileBytes,
+                              nk * kATileBytes, &ctl.full[st], kEvictFirst);
+            };
+            auto load_b = [&](const Seg& sg, int kb, int nk, int st) {
+                const int rows = PAIR ? sg.Nm / 2 : sg.N;
+                const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
+                for (int q = 0; q < nk; ++q) {
+                    uint8_t* b = smB + st * b_stage_bytes + q * b_kb_bytes;
+                    int row = sg.b_row + rank * rows;
+                    const int xk = (kb + q) * bk_elems;
+                    for (int j = 0; j < n64; ++j, row += 64, b += 64 * kRowBytes) {
+                        if constexpr (PAIR)
+                            tma_load_2d_pair(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
+                        else
+                            tma_load_2d(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
+                    }
+                    for (int j = 0; j < n16; ++j, row += 16, b += 16 * kRowBytes) {
+                        if constexpr (PAIR)
+                            tma_load_2d_pair(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
+                        else
+                            tma_load_2d(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
+                    }
+                }
+            };
             // Stages whose weight tiles are issued before the wait for the
             // previous kernel; their activation rows follow after it.
             int early = 0;
@@ -395,17 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Cursor cur = cursor();
                 int u, kb0, kb1;
                 while (early < S && cur.next(u, kb0, kb1)) {
-                    const Seg s = make_seg(ctl, g, u, kb0, kb1);
-                    const uint8_t* a = g.a_tiles +
-                                       (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
-                    const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
-                    for (int kb = s.kb0; kb < s.kb1 && early < S; kb += KPS, ++early) {
-                        const int nk = min(KPS, s.kb1 - kb);
-                        mbar_arrive_expect_tx(&ctl.full[early],
-                                              nk * (kATileBytes + (n64 * 64 + n16 * 16) * kRowBytes));
-                        bulk_load(smA + early * a_stage_bytes,
-                                  a + static_cast<size_t>(kb) * kTileBytes, nk * kATileBytes,
-                                  &ctl.full[early], kEvictFirst);
+                    const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
+                    for (int kb = sg.kb0; kb < sg.kb1 && early < S; kb += KPS, ++early) {
+                        const int nk = min(KPS, sg.kb1 - kb);
+                        if (rank == 0) mbar_arrive_expect_tx(&ctl.full[early], stage_bytes(sg, nk));
+                        load_a(sg, kb, nk, early);
                     }
                 }
             }
@@ -414,15 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             Cursor cur = cursor();
             int u, kb0, kb1;
             while (active && cur.next(u, kb0, kb1)) {
-                const Seg s = make_seg(ctl, g, u, kb0, kb1);
-                const uint8_t* a = g.a_tiles +
-                                   (static_cast<size_t>(s.e * g.MT + s.m) * g.KB) * kTileBytes;
-                const int n64 = s.N >> 6, n16 = (s.N & 63) >> 4;
-                const uint32_t kb_bytes = kATileBytes + (n64 * 64 + n16 * 16) * kRowBytes;
+                const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
                 bool ok = true;
-                for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
+                for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
                     const int st = it % S;
-                    const int nk = min(KPS, s.kb1 - kb);
+                    const int nk = min(KPS, sg.kb1 - kb);
                     if (it >= static_cast<uint32_t>(early)) {
                         const uint32_t par = ((it / S) & 1u) ^ 1u;
                         if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
@@ -430,20 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&ctl.full[st], nk * kb_bytes);
-                        bulk_load(smA + st * a_stage_bytes,
-                                  a + static_cast<size_t>(kb) * kTileBytes, nk * kATileBytes,
-                                  &ctl.full[st], kEvictFirst);
+                        if (rank == 0) mbar_arrive_expect_tx(&ctl.full[st], stage_bytes(sg, nk));
+                        load_a(sg, kb, nk, st);
                     }
-                    for (int q = 0; q < nk; ++q) {
-                        uint8_t* b = smB + st * b_stage_bytes + q * b_kb_bytes;
-                        int row = s.b_row;
-                        const int xk = (kb + q) * bk_elems;
-                        for (int j = 0; j < n64; ++j, row += 64, b += 64 * kRowBytes)
-                            tma_load_2d(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
-                        for (int j = 0; j < n16; ++j, row += 16, b += 16 * kRowBytes)
-                            tma_load_2d(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
-                    }
+                    load_b(sg, kb, nk, st);
                 }
                 if (!ok) break;
             }
@@ -452,13 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0 && active) {
+        if (lane == 0 && active && rank == 0) {
             uint32_t it = 0, si = 0;
             bool ok = true;
             Cursor cur = cursor();
             int u, kb0, kb1;
             for (; ok && cur.next(u, kb0, kb1); ++si) {
-                const Seg s = make_seg(ctl, g, u, kb0, kb1);
+                const Seg s = make_seg<PAIR>(ctl, g, u, kb0, kb1);
                 const int acc = si & 1;
                 if (!mbar_wait(&ctl.tempty[acc], ((si >> 1) & 1u) ^ 1u, &ctl.abort)) {
                     raise_abort(ctl, g.status);
@@ -466,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * g.nmax;
-                const uint32_t idesc = make_idesc<FP8>(kBM, s.N);
+                const uint32_t idesc = make_idesc<FP8>(PAIR ? 2 * kBM : kBM, s.Nm);
                 for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
                     const int st = it % S;
                     const int nk = min(KPS, s.kb1 - kb);
@@ -482,15 +522,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t bd =
                             sw128_desc(smem_u32(smB + st * b_stage_bytes + q * b_kb_bytes));
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc,
-                                      (kb > s.kb0 || q > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t accum = (kb > s.kb0 || q > 0 || kk > 0) ? 1u : 0u;
+                            if constexpr (PAIR)
+                                umma_pair<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
+                            else
+                                umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
+                        }
                     }
                     ctl.mma_issued = 1;
-                    umma_commit(&ctl.empty[st]);
+                    if constexpr (PAIR) umma_commit_pair(&ctl.empty[st]);
+                    else umma_commit(&ctl.empty[st]);
                 }
                 if (!ok) break;
-                umma_commit(&ctl.tfull[acc]);
+                if constexpr (PAIR) umma_commit_pair(&ctl.tfull[acc]);
+                else umma_commit(&ctl.tfull[acc]);
             }
             ctl.mma_pos = it;
         }
@@ -500,6 +546,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;                     // TMEM lane quarter
         const int half = (warp - kEpiWarp0) >> 2;   // which chunks: c0 = 16*(2j + half)
         const int row = 32 * q + lane;              // accumulator row = TMEM lane
+        const int slot_cta = PAIR ? 2 * cta + rank : cta;   // this CTA's partial slots
+        // release of an accumulator: one arrival per warp, on the rank-0 CTA
+        auto release = [&](int acc) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_leader(&ctl.tempty[acc]);
+                else mbar_arrive(&ctl.tempty[acc]);
+            }
+        };
         float act_scale = 1.0f;
         if constexpr (FP8) act_scale = fp8_scale_from_amax(__ldcg(g.act_amax));
         float amax = 0.0f;
@@ -507,8 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         Cursor cur = cursor();
         int u, kb0, kb1;
         for (; active && cur.next(u, kb0, kb1); ++si) {
-            const Seg s = make_seg(ctl, g, u, kb0, kb1);
+            const Seg s = make_seg<PAIR>(ctl, g, u, kb0, kb1);
             const int acc = si & 1;
+            const int m_own = PAIR ? 2 * s.m + rank : s.m;   // this CTA's 128-row weight tile
             // per-unit constants: FP8 dequant factor of this row, routing weights
             float sw = 1.0f;
             if constexpr (FP8)
@@ -535,16 +592,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
                     tmem_ld16(taddr + c0, v);
-                    epilogue_chunk<FP8, EPI>(g, s, c0, v, sw, wreg, staging, amax);
+                    epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, staging, amax);
                 }
-                tc_fence_before();
-                mbar_arrive(&ctl.tempty[acc]);
+                release(acc);
             } else {
                 const long long X0 = static_cast<long long>(s.u - sc.unit0) * g.KB;
                 const int cf = owner_cta(X0, sc.L, sc.Gsk);
                 const int cl = owner_cta(X0 + g.KB - 1, sc.L, sc.Gsk);
                 const long long slot_elems = static_cast<long long>(kBM) * g.nmax;
-                float* mine = g.partials + (2LL * cta + (cta == cf ? 1 : 0)) * slot_elems +
+                float* mine = g.partials + (2LL * slot_cta + (cta == cf ? 1 : 0)) * slot_elems +
                               static_cast<long long>(row) * g.nmax;
                 for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
@@ -554,12 +610,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 4; ++i)
                         p4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
-                tc_fence_before();
-                mbar_arrive(&ctl.tempty[acc]);
+                release(acc);
                 __threadfence();
                 named_bar_epi();
+                const int ctr = PAIR ? 2 * cf + rank : cf;
                 if (threadIdx.x == kEpiWarp0 * 32) {
-                    const int old = atomicAdd(&g.counters[cf], 1);
+                    const int old = atomicAdd(&g.counters[ctr], 1);
                     ctl.flag = (old == cl - cf) ? 1 : 0;
                 }
                 named_bar_epi();
@@ -572,15 +628,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) v[i] = 0.0f;
                         for (int cc = cf; cc <= cl; ++cc) {
+                            const int cc_cta = PAIR ? 2 * cc + rank : cc;
                             const float* p = g.partials +
-                                             (2LL * cc + (cc == cf ? 1 : 0)) * slot_elems +
+                                             (2LL * cc_cta + (cc == cf ? 1 : 0)) * slot_elems +
                                              static_cast<long long>(row) * g.nmax + c0;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i);
                         }
-                        epilogue_chunk<FP8, EPI>(g, s, c0, v, sw, wreg, staging, amax);
+                        epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, staging, amax);
                     }
-                    if (threadIdx.x == kEpiWarp0 * 32) g.counters[cf] = 0;
+                    if (threadIdx.x == kEpiWarp0 * 32) g.counters[ctr] = 0;
                 }
             }
         }
@@ -596,18 +653,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*reinterpret_cast<volatile int*>(&ctl.abort)) {
         // Drain: wait (bounded) for this CTA's own MMAs and copies in flight.
         if (warp == 1 && lane == 0 && ctl.mma_issued) {
-            umma_commit(&ctl.drain);
+            if constexpr (PAIR) umma_commit_pair_local(&ctl.drain);
+            else umma_commit(&ctl.drain);
             mbar_wait(&ctl.drain, 0, nullptr, kDrainLimitNs);
         }
-        if (warp == 0 && lane == 0) {
+        // a pair's copies all complete on the rank-0 CTA's barriers
+        if (warp == 0 && lane == 0 && rank == 0) {
             for (uint32_t it = ctl.mma_pos; it < ctl.prod_pos; ++it)
                 mbar_wait(&ctl.full[it % S], (it / S) & 1u, nullptr, kDrainLimitNs);
         }
         __syncthreads();
     }
+    // neither CTA of a pair frees its TMEM before the pair's MMAs, copies
+    // and epilogues are all done
+    if constexpr (PAIR) cluster_sync();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, g.tmem_cols);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, g.tmem_cols);
+        else tmem_dealloc(tmem_base, g.tmem_cols);
     }
 }
 
@@ -647,17 +710,48 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int K, long rows, int b
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP8, int EPI>
-cudaError_t launch_t(const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& g, int grid,
-                     int smem, cudaStream_t s) {
-    auto kern = grouped_gemm_kernel<FP8, EPI>;
-    // Every launch asks for at most kSmemCap - sizeof(Ctl) - 1024 bytes (see
-    // the stage count below); the 1 KB margin covers the compiler's padding
-    // of the static shared block.
+// Weight tiles viewed as rows of 128 bytes (16 KB tile = 128 rows), copied
+// verbatim (the tiles are already swizzled): boxes of kps tiles.
+bool make_tile_map(CUtensorMap* m, const void* ptr, long tiles, int kps) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kTileRowBytes),
+                                static_cast<cuuint64_t>(tiles) * kTileRows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kTileRowBytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileRowBytes),
+                               static_cast<cuuint32_t>(kps * kTileRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP8, int EPI, bool PAIR>
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b64, const CUtensorMap& b16,
+                     const GemmArgs& g, int grid, int smem, cudaStream_t s) {
+    auto kern = grouped_gemm_kernel<FP8, EPI, PAIR>;
+    // Every launch asks for at most kDynSmemMax bytes (see the stage count
+    // below); the 1 KB margin in it covers the compiler's padding of the
+    // static shared block.
     static cudaError_t attr = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmemMax);
     if (attr != cudaSuccess) return attr;
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, b64, b16, g);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = PAIR ? 2 : 1;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = PAIR ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, b64, b16, g);
 }
 
 int pow2_at_least(int v) {
@@ -698,14 +792,18 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.nmax = p.nmax;
     g.KB = p.KB;
     g.MT = p.MT;
+    // Large token tiles run on CTA pairs (M = 256 per MMA, each CTA loads
+    // half of every token tile); weight streaming runs one CTA per SM.
+    const bool pair = p.nmax > 64;
+    g.MTu = pair ? (p.MT + 1) / 2 : p.MT;
     g.a_tiles = static_cast<const uint8_t*>(p.weights);
     // Two stages of several k-blocks each: small token tiles (weight
     // streaming) take 4 k-blocks (64 KB weight copies), large ones 2 (32 KB
     // weights + 64 KB activations).  Measured on B200: fewer, larger copies
     // sustain more bandwidth than many 16 KB stages, for both regimes.
     const int kps = p.nmax <= 64 ? 4 : 2;
-    const int max_stages = 2;
-    const int stage_bytes = kps * (kATileBytes + p.nmax * kRowBytes);
+    const int max_stages = pair ? 3 : 2;
+    const int stage_bytes = kps * (kATileBytes + (pair ? p.nmax / 2 : p.nmax) * kRowBytes);
     int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
     if (stages > max_stages) stages = max_stages;
     if (stages < 2) return cudaErrorInvalidValue;
@@ -723,19 +821,29 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.partials = p.partials;
     g.counters = p.counters;
     g.status = p.status;
-    CUtensorMap tb64, tb16;
+    CUtensorMap ta, tb64, tb16;
+    memset(&ta, 0, sizeof(ta));
     if (!make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
         !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16))
         return cudaErrorInvalidValue;
+    if (pair && !make_tile_map(&ta, p.weights, static_cast<long>(p.E) * p.MT * p.KB, kps))
+        return cudaErrorInvalidValue;
     int grid = device_sm_count();
     if (p.max_ctas > 0 && p.max_ctas < grid) grid = p.max_ctas;
+    if (pair) grid = grid < 2 ? 2 : grid & ~1;
     const int smem = 1024 + stages * stage_bytes + kStagingBytes;
-    if (p.fp8) {
-        return p.epi == 0 ? launch_t<true, 0>(tb64, tb16, g, grid, smem, s)
-                          : launch_t<true, 1>(tb64, tb16, g, grid, smem, s);
+    if (pair) {
+        if (p.fp8)
+            return p.epi == 0 ? launch_t<true, 0, true>(ta, tb64, tb16, g, grid, smem, s)
+                              : launch_t<true, 1, true>(ta, tb64, tb16, g, grid, smem, s);
+        return p.epi == 0 ? launch_t<false, 0, true>(ta, tb64, tb16, g, grid, smem, s)
+                          : launch_t<false, 1, true>(ta, tb64, tb16, g, grid, smem, s);
     }
-    return p.epi == 0 ? launch_t<false, 0>(tb64, tb16, g, grid, smem, s)
-                      : launch_t<false, 1>(tb64, tb16, g, grid, smem, s);
+    if (p.fp8)
+        return p.epi == 0 ? launch_t<true, 0, false>(ta, tb64, tb16, g, grid, smem, s)
+                          : launch_t<true, 1, false>(ta, tb64, tb16, g, grid, smem, s);
+    return p.epi == 0 ? launch_t<false, 0, false>(ta, tb64, tb16, g, grid, smem, s)
+                      : launch_t<false, 1, false>(ta, tb64, tb16, g, grid, smem, s);
 }
 
 }  // namespace moe

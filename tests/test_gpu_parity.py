@@ -165,6 +165,20 @@ def test_forward_stream_k_splits(moe, dtype, max_ctas):
     assert_close(out, ref, dtype, f"max_ctas={max_ctas}")
 
 
+@pytest.mark.parametrize("max_ctas", [2, 7, 14, 0])
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_forward_cta_pair_splits(moe, dtype, max_ctas):
+    """Large token tiles run on CTA pairs (M = 256 per MMA): odd weight-tile
+    counts (5 gate/up, 3 down tiles), ragged token tiles and capped grids that
+    split pair units stream-K style."""
+    L = make_layer("tiny", T=600, E=4, k=2, H=384, I=320, seed=6)
+    out, ids, w = run_forward(moe, dtype, L, max_ctas=max_ctas)
+    ids_o, w_o = check_routing(ids, w, L.logits)
+    g, u, d = L.weights_bf16()
+    ref = oracle_layer(dtype, L.x, ids_o, w_o, g, u, d)
+    assert_close(out, ref, dtype, f"pair max_ctas={max_ctas}")
+
+
 @pytest.mark.parametrize("block_m", [16, 32, 64, 128])
 def test_forward_block_m_variants(moe, block_m):
     L = make_layer("tiny", T=50, E=8, k=2, H=256, I=256, seed=9)
