@@ -264,6 +264,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
 template <bool FP8, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB128,
                         const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
     extern __shared__ uint8_t dsmem_raw[];
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (warp == 0 && lane == 0) {
             if constexpr (PAIR) tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB128);
             tma_prefetch_desc(&tmB64);
             tma_prefetch_desc(&tmB16);
         }
@@ -429,11 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto load_b = [&](const Seg& sg, int kb, int nk, int st) {
                 const int rows = PAIR ? sg.Nm / 2 : sg.N;
-                const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
+                const int n128 = rows >> 7, n64 = (rows & 127) >> 6, n16 = (rows & 63) >> 4;
                 for (int q = 0; q < nk; ++q) {
                     uint8_t* b = smB + st * b_stage_bytes + q * b_kb_bytes;
                     int row = sg.b_row + rank * rows;
                     const int xk = (kb + q) * bk_elems;
+                    for (int j = 0; j < n128; ++j, row += 128, b += 128 * kRowBytes) {
+                        if constexpr (PAIR)
+                            tma_load_2d_pair(b, &tmB128, &ctl.full[st], xk, row, kEvictLast);
+                        else
+                            tma_load_2d(b, &tmB128, &ctl.full[st], xk, row, kEvictLast);
+                    }
                     for (int j = 0; j < n64; ++j, row += 64, b += 64 * kRowBytes) {
                         if constexpr (PAIR)
                             tma_load_2d_pair(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
@@ -728,8 +736,9 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, long tiles, int kps) {
 }
 
 template <bool FP8, int EPI, bool PAIR>
-cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b64, const CUtensorMap& b16,
-                     const GemmArgs& g, int grid, int smem, cudaStream_t s) {
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b128, const CUtensorMap& b64,
+                     const CUtensorMap& b16, const GemmArgs& g, int grid, int smem,
+                     cudaStream_t s) {
     auto kern = grouped_gemm_kernel<FP8, EPI, PAIR>;
     // Every launch asks for at most kDynSmemMax bytes (see the stage count
     // below); the 1 KB margin in it covers the compiler's padding of the
@@ -751,7 +760,7 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b64, const CUtenso
     at[1].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = PAIR ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, b64, b16, g);
+    return cudaLaunchKernelEx(&cfg, kern, a, b128, b64, b16, g);
 }
 
 int pow2_at_least(int v) {
@@ -821,9 +830,10 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.partials = p.partials;
     g.counters = p.counters;
     g.status = p.status;
-    CUtensorMap ta, tb64, tb16;
+    CUtensorMap ta, tb128, tb64, tb16;
     memset(&ta, 0, sizeof(ta));
-    if (!make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
+    if (!make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
+        !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
         !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16))
         return cudaErrorInvalidValue;
     if (pair && !make_tile_map(&ta, p.weights, static_cast<long>(p.E) * p.MT * p.KB, kps))
@@ -834,16 +844,16 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     const int smem = 1024 + stages * stage_bytes + kStagingBytes;
     if (pair) {
         if (p.fp8)
-            return p.epi == 0 ? launch_t<true, 0, true>(ta, tb64, tb16, g, grid, smem, s)
-                              : launch_t<true, 1, true>(ta, tb64, tb16, g, grid, smem, s);
-        return p.epi == 0 ? launch_t<false, 0, true>(ta, tb64, tb16, g, grid, smem, s)
-                          : launch_t<false, 1, true>(ta, tb64, tb16, g, grid, smem, s);
+            return p.epi == 0 ? launch_t<true, 0, true>(ta, tb128, tb64, tb16, g, grid, smem, s)
+                              : launch_t<true, 1, true>(ta, tb128, tb64, tb16, g, grid, smem, s);
+        return p.epi == 0 ? launch_t<false, 0, true>(ta, tb128, tb64, tb16, g, grid, smem, s)
+                          : launch_t<false, 1, true>(ta, tb128, tb64, tb16, g, grid, smem, s);
     }
     if (p.fp8)
-        return p.epi == 0 ? launch_t<true, 0, false>(ta, tb64, tb16, g, grid, smem, s)
-                          : launch_t<true, 1, false>(ta, tb64, tb16, g, grid, smem, s);
-    return p.epi == 0 ? launch_t<false, 0, false>(ta, tb64, tb16, g, grid, smem, s)
-                      : launch_t<false, 1, false>(ta, tb64, tb16, g, grid, smem, s);
+        return p.epi == 0 ? launch_t<true, 0, false>(ta, tb128, tb64, tb16, g, grid, smem, s)
+                          : launch_t<true, 1, false>(ta, tb128, tb64, tb16, g, grid, smem, s);
+    return p.epi == 0 ? launch_t<false, 0, false>(ta, tb128, tb64, tb16, g, grid, smem, s)
+                      : launch_t<false, 1, false>(ta, tb128, tb64, tb16, g, grid, smem, s);
 }
 
 }  // namespace moe
