@@ -60,7 +60,7 @@ constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
 struct GemmArgs {
     int E, Mw, K, KB, MT, MTu, Mvalid;   // MTu: weight tiles per unit step (MT, or pairs)
-    int nmax, stages, kps, tmem_cols;
+    int nmax, stages, tmem_cols;
     const uint8_t* a_tiles;
     int ldo;
     void* out;
@@ -274,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     // stage = kps consecutive k-blocks: A kps*16 KB (one bulk copy), B kps
     // slots of nmax rows x 128 B
-    const int KPS = g.kps;
+    // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
+    constexpr int KPS = PAIR ? 2 : 4;
     const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
     const int a_stage_bytes = KPS * kATileBytes;
     // a pair member holds half of each token tile
@@ -475,14 +476,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             pdl_trigger();
             Cursor cur = cursor();
             int u, kb0, kb1;
+            int st = 0;
+            uint32_t par = 1;   // parity of the empty-barrier phase the next refill waits for
             while (active && cur.next(u, kb0, kb1)) {
                 const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
                 bool ok = true;
                 for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
-                    const int st = it % S;
                     const int nk = min(KPS, sg.kb1 - kb);
                     if (it >= static_cast<uint32_t>(early)) {
-                        const uint32_t par = ((it / S) & 1u) ^ 1u;
                         if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
                             raise_abort(ctl, g.status);
                             ok = false;
@@ -492,6 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         load_a(sg, kb, nk, st);
                     }
                     load_b(sg, kb, nk, st);
+                    if (++st == S) {
+                        st = 0;
+                        par ^= 1u;
+                    }
                 }
                 if (!ok) break;
             }
@@ -501,10 +506,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && active && rank == 0) {
-            uint32_t it = 0, si = 0;
+            // The issue loop is kept short: one thread feeds the tensor core,
+            // and at N <= 128 an MMA takes only tens of cycles.  Stage index
+            // and phase advance incrementally, and descriptors advance by
+            // adding (byte offset >> 4) to their start-address field.
+            const uint64_t a_desc0 = sw128_desc(smem_u32(smA));
+            const uint64_t b_desc0 = sw128_desc(smem_u32(smB));
+            const uint32_t a_step = static_cast<uint32_t>(a_stage_bytes) >> 4;
+            const uint32_t b_step = static_cast<uint32_t>(b_stage_bytes) >> 4;
+            const uint32_t b_kb = static_cast<uint32_t>(b_kb_bytes) >> 4;
+            uint64_t ast = a_desc0, bst = b_desc0;
+            int st = 0;
+            uint32_t ph = 0, it = 0, si = 0;
             bool ok = true;
             Cursor cur = cursor();
             int u, kb0, kb1;
+            ctl.mma_issued = 1;
             for (; ok && cur.next(u, kb0, kb1); ++si) {
                 const Seg s = make_seg<PAIR>(ctl, g, u, kb0, kb1);
                 const int acc = si & 1;
@@ -516,31 +533,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d = tmem_base + acc * g.nmax;
                 const uint32_t idesc = make_idesc<FP8>(PAIR ? 2 * kBM : kBM, s.Nm);
                 for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
-                    const int st = it % S;
-                    const int nk = min(KPS, s.kb1 - kb);
-                    if (!mbar_wait(&ctl.full[st], (it / S) & 1u, &ctl.abort)) {
+                    const int nk = s.kb1 - kb;
+                    if (!mbar_wait(&ctl.full[st], ph, &ctl.abort)) {
                         raise_abort(ctl, g.status);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    for (int q = 0; q < nk; ++q) {
-                        const uint64_t ad =
-                            sw128_desc(smem_u32(smA + st * a_stage_bytes + q * kATileBytes));
-                        const uint64_t bd =
-                            sw128_desc(smem_u32(smB + st * b_stage_bytes + q * b_kb_bytes));
+                    const uint32_t first = kb == s.kb0 ? 0u : 1u;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t accum = (kb > s.kb0 || q > 0 || kk > 0) ? 1u : 0u;
-                            if constexpr (PAIR)
-                                umma_pair<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
-                            else
-                                umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
+                    for (int q = 0; q < KPS; ++q) {
+                        if (q == 0 || q < nk) {
+                            const uint64_t ad = ast + static_cast<uint32_t>(q * (kATileBytes >> 4));
+                            const uint64_t bd = bst + static_cast<uint32_t>(q) * b_kb;
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t accum = (q | kk) ? 1u : first;
+                                if constexpr (PAIR)
+                                    umma_pair<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
+                                else
+                                    umma<FP8>(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
+                            }
                         }
                     }
-                    ctl.mma_issued = 1;
                     if constexpr (PAIR) umma_commit_pair(&ctl.empty[st]);
                     else umma_commit(&ctl.empty[st]);
+                    if (++st == S) {
+                        st = 0;
+                        ph ^= 1u;
+                        ast = a_desc0;
+                        bst = b_desc0;
+                    } else {
+                        ast += a_step;
+                        bst += b_step;
+                    }
                 }
                 if (!ok) break;
                 if constexpr (PAIR) umma_commit_pair(&ctl.tfull[acc]);
@@ -608,15 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int cf = owner_cta(X0, sc.L, sc.Gsk);
                 const int cl = owner_cta(X0 + g.KB - 1, sc.L, sc.Gsk);
                 const long long slot_elems = static_cast<long long>(kBM) * g.nmax;
-                float* mine = g.partials + (2LL * slot_cta + (cta == cf ? 1 : 0)) * slot_elems +
-                              static_cast<long long>(row) * g.nmax;
+                // partial tiles are column-major (element (row, col) at
+                // col * 128 + row): a warp's 32 rows form one 128-byte line
+                float* mine = g.partials + (2LL * slot_cta + (cta == cf ? 1 : 0)) * slot_elems + row;
                 for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
                     tmem_ld16(taddr + c0, v);
-                    float4* p4 = reinterpret_cast<float4*>(mine + c0);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        p4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    for (int i = 0; i < 16; ++i) __stcg(mine + (c0 + i) * kBM, v[i]);
                 }
                 release(acc);
                 __threadfence();
@@ -639,9 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int cc_cta = PAIR ? 2 * cc + rank : cc;
                             const float* p = g.partials +
                                              (2LL * cc_cta + (cc == cf ? 1 : 0)) * slot_elems +
-                                             static_cast<long long>(row) * g.nmax + c0;
+                                             c0 * kBM + row;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i);
+                            for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i * kBM);
                         }
                         epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, staging, amax);
                     }
@@ -810,14 +835,13 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     // streaming) take 4 k-blocks (64 KB weight copies), large ones 2 (32 KB
     // weights + 64 KB activations).  Measured on B200: fewer, larger copies
     // sustain more bandwidth than many 16 KB stages, for both regimes.
-    const int kps = p.nmax <= 64 ? 4 : 2;
+    const int kps = pair ? 2 : 4;   // the kernel's KPS
     const int max_stages = pair ? 3 : 2;
     const int stage_bytes = kps * (kATileBytes + (pair ? p.nmax / 2 : p.nmax) * kRowBytes);
     int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
     if (stages > max_stages) stages = max_stages;
     if (stages < 2) return cudaErrorInvalidValue;
     g.stages = stages;
-    g.kps = kps;
     g.tmem_cols = pow2_at_least(2 * p.nmax);
     g.ldo = p.ldo;
     g.out = p.out;
