@@ -41,9 +41,10 @@ WORKLOADS = {
     "skewed": dict(cfg="skewed", dtype=0, bound="tensor"),
 }
 NBATCH = 4
+GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
 # DRAM bytes (read + write) of one gate/up launch from an ncu capture of the
 # same kernel build, keyed by (workload, T); None until captured.
-TRAFFIC = {("decode", 64): 1888433920}
+TRAFFIC = {("decode", 64): 1887167120, ("prefill", 4096): 1378159440}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 
 
@@ -245,8 +246,16 @@ def run_native(args):
             ids, _ = moe.route_topk(lg, k)
             active[T].append(int(torch.unique(ids).numel()))
 
-    def step(i, ev=None):
+    # Small token counts (T <= 64) run as CUDA graphs, one per rotating batch:
+    # there the layer is a short chain of short kernels and the launch cost
+    # on the host would otherwise show.  Larger T launch directly.
+    graphs, graph_note = {}, None
+
+    def step(i, ev=None, direct=False):
         for T in Ts:
+            if T in graphs and ev is None and not direct:
+                graphs[T][i % NBATCH].replay()
+                continue
             x, lg = dev_in[T][i % NBATCH]
             layer(x, lg, out=outs[T], events=None if ev is None else ev[T])
 
@@ -255,6 +264,29 @@ def run_native(args):
     torch.cuda.synchronize()
     if layer.check() != 0:
         raise RuntimeError("device status word reports a fault")
+    if not args.no_graphs:
+        try:
+            for T in Ts:
+                if T > GRAPH_MAX_T:
+                    continue
+                gl = []
+                for b in range(NBATCH):
+                    x, lg = dev_in[T][b]
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        layer(x, lg, out=outs[T])
+                    gl.append(g)
+                graphs[T] = gl
+            for i in range(args.warmup):
+                step(i)
+            torch.cuda.synchronize()
+            if layer.check() != 0:
+                raise RuntimeError("device status word reports a fault")
+        except RuntimeError as ex:
+            if "status word" in str(ex):
+                raise
+            graphs.clear()
+            graph_note = "graph capture failed, direct launches: " + str(ex).splitlines()[0]
 
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -304,7 +336,19 @@ def run_native(args):
     layer_ms = {T: statistics.mean([sum(stage[T][s][j] for s in range(6))
                                     for j in range(args.steps)]) for T in Ts}
     # whole-layer time of each T inside the headline region, from a third pass
-    # of single-T steps timed without stage events
+    # of single-T steps timed without stage events (graph replays where the
+    # headline uses them; the direct-launch time is reported beside it)
+    layer_graph_ms = {}
+    for T in graphs:
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[T][i % NBATCH].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        layer_graph_ms[T] = e0.elapsed_time(e1) / args.steps
     layer_pdl_ms = {}
     for T in Ts:
         e0 = torch.cuda.Event(enable_timing=True)
@@ -350,17 +394,18 @@ def run_native(args):
         a = statistics.mean(active[T])
         layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
         layer_flops = 6.0 * T * k * H * I
-        per_T[str(T)] = {"layer_us": round(1e3 * layer_pdl_ms[T], 2),
-                         "layer_tflops": round(layer_flops / (layer_pdl_ms[T] / 1e3) / 1e12, 1),
-                         "layer_tensor_frac": round(layer_flops / (layer_pdl_ms[T] / 1e3) / 1e12
-                                                    / tpeak, 4),
+        lt = layer_graph_ms.get(T, layer_pdl_ms[T])
+        per_T[str(T)] = {"layer_us": round(1e3 * lt, 2),
+                         "layer_us_direct": round(1e3 * layer_pdl_ms[T], 2),
+                         "cuda_graph": T in graphs,
+                         "layer_tflops": round(layer_flops / (lt / 1e3) / 1e12, 1),
+                         "layer_tensor_frac": round(layer_flops / (lt / 1e3) / 1e12 / tpeak, 4),
                          "layer_us_staged": round(1e3 * layer_ms[T], 2),
                          "gate_up_us": round(1e3 * gu_ms[T], 2),
                          "down_us": round(1e3 * dn_ms[T], 2),
                          "active_experts": a,
-                         "layer_hbm_gbs": round(layer_bytes / (layer_pdl_ms[T] / 1e3) / 1e9, 1),
-                         "layer_hbm_frac": round(layer_bytes / (layer_pdl_ms[T] / 1e3) / 1e9 / hbm,
-                                                 4)}
+                         "layer_hbm_gbs": round(layer_bytes / (lt / 1e3) / 1e9, 1),
+                         "layer_hbm_frac": round(layer_bytes / (lt / 1e3) / 1e9 / hbm, 4)}
 
     # end to end through the public call, host buffers, copies in the timed region
     e2e = None
@@ -414,6 +459,7 @@ def run_native(args):
                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                            "l2": "inputs larger than L2: expert weights "
                                  f"{3 * E * H * I * wb / 1e9:.2f} GB, {NBATCH} rotating batches",
+                           "cuda_graphs": sorted(graphs) if graphs else (graph_note or "none"),
                            "per_T": per_T},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clk.summary()}
@@ -432,6 +478,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="launch every T directly (no CUDA graphs for T <= 64)")
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--Ts", default="", help="comma-separated subset of the token counts")
     args = ap.parse_args()
