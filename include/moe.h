@@ -124,7 +124,7 @@ MOE_API moe_status moe_align_permute(const int32_t* ids, int T, int k, int E, in
  * Arguments and outputs are those of moe_align_permute without ws/ws_bytes.
  * Its scratch is a fixed 256 KB device array inside the library (65536
  * int32 counters, held on every GPU that loads the library until exit), so
- * ceil(T*k/2048) * E must not exceed 65536; larger problems return
+ * for T*k > 2048, ceil(T*k/512) * E must not exceed 65536; larger problems return
  * MOE_ERR_WORKSPACE with nothing launched.  The first call on a device looks
  * up the array's address for that device; make it before any stream capture.
  * All calls share the array: each overwrites what it reads, but calls that

@@ -9,7 +9,8 @@
 // a2: the "data reordering" of "Az AWS új MoE-optimalizációkkal gyorsítja a
 //     SageMaker AI-t", § "A fused MoE a számítási folyamat több lépését
 //     egyesíti": a stable counting sort of the assignments by expert, with no
-//     atomics.  Assignments are cut into chunks of 2048 (a slice per warp); each
+//     atomics.  Assignments are cut into chunks (all of them, up to 2048, in
+//     the single-CTA kernel; 512 per CTA otherwise), a slice per warp; each
 //     warp counts its slice with __match_any_sync (the lowest lane of each
 //     group of equal ids adds the group size to the warp's private histogram),
 //     per-expert prefix sums over (chunk, warp) give every warp a start
@@ -30,6 +31,11 @@ constexpr int kThreads = 256;        // multi-CTA kernels: 8 warps
 constexpr int kSmallThreads = 512;   // single-CTA kernel: 16 warps
 constexpr int kStageFloats = 4096;   // logits staged in smem by the single-CTA kernel
 constexpr unsigned kFull = 0xffffffffu;
+// Multi-CTA permutation: assignments per chunk (one CTA of 8 warps, 64 per
+// warp).  Small chunks give a few-thousand-token batch dozens of CTAs; the
+// per-chunk counters (nchunks x E) are scanned in batches of independent loads.
+constexpr int kPermChunk = 512;
+constexpr int kScanBatch = 16;
 
 __device__ __forceinline__ bool beats(float a, int ia, float b, int ib) {
     const bool na = isnan(a), nb = isnan(b);
@@ -41,9 +47,11 @@ __device__ __forceinline__ bool beats(float a, int ia, float b, int ib) {
     return ia < ib;
 }
 
-// Top-k of row[0..E) by one warp (row in global or shared memory).  Lane 0
-// writes the ids in selection order; the weights are a softmax over the
-// selected logits, re-read through the ids.
+// Top-k of row[0..E) by one warp (row in global or shared memory).  The
+// j-th selection (id and logit, known to every lane after the arg-max) is kept
+// in registers of lane j % 32, slot j / 32; the weights are a softmax over the
+// selected logits, summed per lane in ascending j and then across the warp.
+// ids and w are written once at the end, lane j for entry j.
 template <int EPL>
 __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w) {
     const int lane = threadIdx.x & 31;
@@ -54,6 +62,13 @@ __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w
         const int e = lane + 32 * i;
         v[i] = e < E ? row[e] : 0.0f;
         if (e >= E) taken |= 1u << i;
+    }
+    float sv[EPL];
+    int si[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        sv[i] = 0.0f;
+        si[i] = 0;
     }
     float m = 0.0f;
     for (int j = 0; j < k; ++j) {
@@ -78,15 +93,30 @@ __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w
             }
         }
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == 0) ids[j] = bi;
+        if ((j & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == (j >> 5)) {
+                    sv[i] = bv;
+                    si[i] = bi;
+                }
+        }
         if (j == 0) m = bv;
     }
-    __syncwarp();
     float z = 0.0f;
-    for (int j = lane; j < k; j += 32) z += expf(row[ids[j]] - m);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i < k) z += expf(sv[i] - m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
-    for (int j = lane; j < k; j += 32) w[j] = expf(row[ids[j]] - m) / z;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int j = lane + 32 * i;
+        if (j < k) {
+            ids[j] = si[i];
+            w[j] = expf(sv[i] - m) / z;
+        }
+    }
     __syncwarp();
 }
 
@@ -108,10 +138,10 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // hist[w][e] += number of assignments of warp w's slice of the chunk routed to e
-template <int NW>
+template <int NW, int CHUNK>
 __device__ void chunk_histogram(const int32_t* ids, long A, long chunk_base, int E,
                                 int (*hist)[kMaxExperts], int32_t* status) {
-    constexpr int kPerWarp = kChunk / NW;
+    constexpr int kPerWarp = CHUNK / NW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long wbase = chunk_base + static_cast<long>(warp) * kPerWarp;
     for (int r = 0; r < kPerWarp / 32; ++r) {
@@ -131,10 +161,10 @@ __device__ void chunk_histogram(const int32_t* ids, long A, long chunk_base, int
 }
 
 // Places the warp's slice: base[w][e] holds the next free slot of expert e.
-template <int NW>
+template <int NW, int CHUNK>
 __device__ void chunk_scatter(const int32_t* ids, long A, long chunk_base, int E,
                               int (*base)[kMaxExperts], int32_t* sorted_ids, int32_t* inv_perm) {
-    constexpr int kPerWarp = kChunk / NW;
+    constexpr int kPerWarp = CHUNK / NW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long wbase = chunk_base + static_cast<long>(warp) * kPerWarp;
     for (int r = 0; r < kPerWarp / 32; ++r) {
@@ -244,7 +274,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     }
     for (int i = threadIdx.x; i < NW * kMaxExperts; i += kSmallThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    chunk_histogram<NW>(ids, A, 0, E, hist, status);
+    chunk_histogram<NW, kChunk>(ids, A, 0, E, hist, status);
     __syncthreads();
     const int e = threadIdx.x;
     int c = 0;
@@ -263,7 +293,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     const int total = tmp[NW];
     __syncthreads();
     fill_tail<kSmallThreads>(total, block_m, capacity, sorted_ids, tiles);
-    chunk_scatter<NW>(ids, A, 0, E, hist, sorted_ids, inv_perm);
+    chunk_scatter<NW, kChunk>(ids, A, 0, E, hist, sorted_ids, inv_perm);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -275,7 +305,8 @@ __global__ void __launch_bounds__(kThreads)
     pdl_trigger();
     for (int i = threadIdx.x; i < NW * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    chunk_histogram<NW>(ids, A, static_cast<long>(blockIdx.x) * kChunk, E, hist, status);
+    chunk_histogram<NW, kPermChunk>(ids, A, static_cast<long>(blockIdx.x) * kPermChunk, E, hist,
+                                    status);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int c = 0;
@@ -295,10 +326,17 @@ __global__ void __launch_bounds__(kThreads)
     const int e = threadIdx.x;
     int run = 0;
     if (e < E)
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = chunk_counts[static_cast<long>(c) * E + e];
-            chunk_counts[static_cast<long>(c) * E + e] = run;
-            run += v;
+        for (int c0 = 0; c0 < nchunks; c0 += kScanBatch) {
+            // the batch's loads are independent: issue them all, then scan
+            int v[kScanBatch];
+#pragma unroll
+            for (int i = 0; i < kScanBatch; ++i)
+                v[i] = c0 + i < nchunks ? chunk_counts[static_cast<long>(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kScanBatch; ++i) {
+                if (c0 + i < nchunks) chunk_counts[static_cast<long>(c0 + i) * E + e] = run;
+                run += v[i];
+            }
         }
     finish_offsets<kThreads>(run, E, block_m, counts, offsets, sorted_ids, tiles, num_tiles, tmp);
     const int total = tmp[NW];
@@ -317,8 +355,8 @@ __global__ void __launch_bounds__(kThreads)
     pdl_trigger();
     for (int i = threadIdx.x; i < NW * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    const long base = static_cast<long>(blockIdx.x) * kChunk;
-    chunk_histogram<NW>(ids, A, base, E, hist, nullptr);
+    const long base = static_cast<long>(blockIdx.x) * kPermChunk;
+    chunk_histogram<NW, kPermChunk>(ids, A, base, E, hist, nullptr);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int run = offsets[e] + chunk_prefix[static_cast<long>(blockIdx.x) * E + e];
@@ -329,14 +367,18 @@ __global__ void __launch_bounds__(kThreads)
         }
     }
     __syncthreads();
-    chunk_scatter<NW>(ids, A, base, E, hist, sorted_ids, inv_perm);
+    chunk_scatter<NW, kPermChunk>(ids, A, base, E, hist, sorted_ids, inv_perm);
 }
 
 int epl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 
 }  // namespace
 
-int permute_chunks(long A) { return static_cast<int>((A + kChunk - 1) / kChunk); }
+// 1 when the single-CTA kernel handles all A assignments, else the number of
+// chunks (and per-chunk counter rows) of the multi-CTA path.
+int permute_chunks(long A) {
+    return A <= kChunk ? 1 : static_cast<int>((A + kPermChunk - 1) / kPermChunk);
+}
 
 bool fused_route_permute_ok(int T, int k) {
     return T <= kSmallT && static_cast<long>(T) * k <= kChunk;

@@ -53,7 +53,8 @@ def test_capacity_matches_oracle(L, T, k, E, bm):
 def test_workspace_sizes(L):
     lib = L.lib()
     assert lib.moe_align_permute_workspace_size(64, 2, 8) == 0       # single chunk
-    assert lib.moe_align_permute_workspace_size(4096, 8, 128) == 16 * 128 * 4
+    assert lib.moe_align_permute_workspace_size(4096, 8, 128) == 64 * 128 * 4   # 512 per chunk
+    assert lib.moe_align_permute_workspace_size(256, 8, 128) == 0                # one CTA up to 2048
     # 16 KB tiles of 128 rows x 128 bytes, padded per expert matrix
     assert lib.moe_packed_weights_size(0, 8, 4096, 14336) == 3 * 8 * 4096 * 14336 * 2
     tiles = 32 * ((2 * 2880 // 128) * 23 + 23 * 23)

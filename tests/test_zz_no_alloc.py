@@ -18,7 +18,7 @@ KEYS = ("counts", "offsets", "sorted_ids", "inv_perm", "tiles", "num_tiles")
 
 def test_noalloc_matches_workspace_entry_twice():
     moe = lib()
-    cases = [(8192, 256, 8, 16, 1.2),   # 32 chunks x 256 experts of built-in scratch
+    cases = [(8192, 256, 8, 16, 1.2),   # 128 chunks x 256 experts of built-in scratch
              (3000, 32, 4, 64, 0.5)]    # fewer experts: stale counters must not leak
     results = []
     for T, E, k, bm, skew in cases:
@@ -34,7 +34,7 @@ def test_noalloc_matches_workspace_entry_twice():
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
     moe = lib()
-    # ceil(T*k/2048) * E > 65536 counters: refused before any launch
+    # ceil(T*k/512) * E > 65536 counters: refused before any launch
     T, k, E = 70000, 8, 256
     ids = torch.zeros((1, 1), dtype=torch.int32, device=DEV)   # never read
     lib_ = moe.lib()
