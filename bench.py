@@ -179,6 +179,16 @@ def oracle_sample(W, dtype, Ts, budget_s=12.0):
     return n / el, oracle.num_threads(), what
 
 
+def aggregate_over_ranks(elapsed_ms, tokens_per_step, steps, world, dist=None, device=None):
+    """Whole-job throughput of a timed region: the slowest rank's time (max over
+    ranks) and the tokens all ranks processed in it.  Returns (ms, tokens/s)."""
+    el = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(el, op=dist.ReduceOp.MAX)
+    ms = float(el.item())
+    return ms, tokens_per_step * steps * world / (ms / 1e3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -307,12 +317,9 @@ def run_native(args):
     elapsed_ms = t_start.elapsed_time(t_end)
     if layer.check() != 0:
         raise RuntimeError("device status word reports a fault")
-    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(el, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(el.item())
     tokens_per_step = sum(Ts)
-    value = tokens_per_step * args.steps * world / (elapsed_ms / 1e3)
+    elapsed_ms, value = aggregate_over_ranks(elapsed_ms, tokens_per_step, args.steps, world,
+                                             dist if world > 1 else None, dev)
 
     # stage region: the same steps with CUDA events recorded between the
     # layer's stages on the launching stream (an event between two kernels
@@ -435,10 +442,9 @@ def run_native(args):
             e2e_step(i)
         a1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
-        if dist:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_per_step * args.steps * world / (float(e_ms.item()) / 1e3),
+        _, e_val = aggregate_over_ranks(a0.elapsed_time(a1), tokens_per_step, args.steps, world,
+                                        dist if world > 1 else None, dev)
+        e2e = {"value": e_val,
                "unit": "tokens/s",
                "h2d_bytes_per_step": sum(T * H * 2 + T * E * 4 for T in Ts),
                "d2h_bytes_per_step": sum(T * H * 2 for T in Ts)}

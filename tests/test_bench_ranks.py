@@ -1,0 +1,59 @@
+"""The multi-rank plumbing of bench.py, on the CPU: the max-over-ranks timing
+reduction over a 2-rank gloo group, and the reference arm's rule that only
+rank 0 works (the other ranks exit 0 at once)."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _rank_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = 10.0 * (rank + 1)             # rank r took 10*(r+1) ms
+        out = bench.aggregate_over_ranks(ms, tokens_per_step=85, steps=4, world=world,
+                                         dist=dist)
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_takes_max_over_ranks_gloo():
+    world, port = 2, 29517
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        ms, value = res[r]
+        assert ms == 20.0                         # the slowest rank's time
+        assert value == pytest.approx(85 * 4 * world / 0.020)
+
+
+def test_aggregate_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    ms, value = bench.aggregate_over_ranks(5.0, 10, 2, 1)
+    assert ms == 5.0 and value == pytest.approx(10 * 2 / 0.005)
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
