@@ -37,31 +37,40 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kPermChunk = 512;
 constexpr int kScanBatch = 16;
 
-__device__ __forceinline__ bool beats(float a, int ia, float b, int ib) {
-    const bool na = isnan(a), nb = isnan(b);
-    if (na || nb) {
-        if (na && nb) return ia < ib;
-        return nb;
-    }
-    if (a != b) return a > b;
-    return ia < ib;
+// Selection order as one 64-bit key, larger first: an order-preserving map of
+// the logit (-0 folded onto +0; NaN below every number) in the high word and
+// the complement of the expert index in the low word (equal logits: the lower
+// index wins).  Key 0 marks an expert already taken or past E.
+__device__ __forceinline__ uint64_t select_key(float f, int e) {
+    uint32_t b = __float_as_uint(f);
+    if (b == 0x80000000u) b = 0u;
+    const uint32_t ord = isnan(f) ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+    return (static_cast<uint64_t>(ord) << 32) | (0xffffffffu - static_cast<uint32_t>(e));
 }
 
-// Top-k of row[0..E) by one warp (row in global or shared memory).  The
-// j-th selection (id and logit, known to every lane after the arg-max) is kept
-// in registers of lane j % 32, slot j / 32; the weights are a softmax over the
-// selected logits, summed per lane in ascending j and then across the warp.
-// ids and w are written once at the end, lane j for entry j.
+// The logit of a key (exact, except -0 reads as +0 and a NaN as the canonical
+// NaN; neither changes exp(l - m)).
+__device__ __forceinline__ float key_value(uint64_t key) {
+    const uint32_t ord = static_cast<uint32_t>(key >> 32);
+    if (ord == 0u) return __uint_as_float(0x7fffffffu);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+}
+
+// Top-k of row[0..E) by one warp (row in global or shared memory).  Each lane
+// keys its E/32 logits once; a selection round is a local max of the lane's
+// keys and a five-step warp max, after which the owning lane clears the
+// winner.  The j-th selection (id and logit) is kept in registers of lane
+// j % 32, slot j / 32; the weights are a softmax over the selected logits,
+// summed per lane in ascending j and then across the warp.  ids and w are
+// written once at the end, lane j for entry j.
 template <int EPL>
 __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w) {
     const int lane = threadIdx.x & 31;
-    float v[EPL];
-    uint32_t taken = 0;
+    uint64_t key[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? row[e] : 0.0f;
-        if (e >= E) taken |= 1u << i;
+        key[i] = e < E ? select_key(row[e], e) : 0ull;
     }
     float sv[EPL];
     int si[EPL];
@@ -72,27 +81,21 @@ __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w
     }
     float m = 0.0f;
     for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int bi = INT_MAX;
+        uint64_t best = key[0];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            if (taken & (1u << i)) continue;
-            const int e = lane + 32 * i;
-            if (bi == INT_MAX || beats(v[i], e, bv, bi)) {
-                bv = v[i];
-                bi = e;
-            }
-        }
+        for (int i = 1; i < EPL; ++i) best = key[i] > best ? key[i] : best;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(kFull, bv, off);
-            const int oi = __shfl_xor_sync(kFull, bi, off);
-            if (oi != INT_MAX && (bi == INT_MAX || beats(ov, oi, bv, bi))) {
-                bv = ov;
-                bi = oi;
-            }
+            const uint64_t o = __shfl_xor_sync(kFull, best, off);
+            best = o > best ? o : best;
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        const int bi = static_cast<int>(0xffffffffu - static_cast<uint32_t>(best));
+        const float bv = key_value(best);
+        if ((bi & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == (bi >> 5)) key[i] = 0ull;
+        }
         if ((j & 31) == lane) {
 #pragma unroll
             for (int i = 0; i < EPL; ++i)
