@@ -46,6 +46,7 @@ GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
 # same kernel build, keyed by (workload, T); None until captured.
 TRAFFIC = {("decode", 64): 1887167120, ("prefill", 4096): 1378159440}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
+SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
 
 
 def describe(name):
@@ -55,14 +56,16 @@ def describe(name):
             f"T={','.join(str(t) for t in c['T'])}")
 
 
-def kernels_per_forward(T, k, fp8):
+def kernels_per_forward(T, k, fp8, H):
     """Kernels one moe_forward launches (the cudaMemsetAsync is not a kernel)."""
     A = T * k
-    if T <= SMALL_T and A <= CHUNK:
+    small = T <= SMALL_T and A <= CHUNK
+    if small:
         n = 1                                   # fused route + permute
     else:
         n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
-    n += 2 if fp8 else 1                        # [amax] + gather
+    n += 1                                      # gather
+    n += 1 if fp8 and not (small and T * H <= SMALL_AMAX) else 0   # amax(x)
     n += 1                                      # gate/up GEMM
     n += 1 if fp8 else 0                        # h quantisation
     n += 2                                      # down GEMM + combine
@@ -454,7 +457,7 @@ def run_native(args):
         v, cores, what = oracle_sample(W, dtype, Ts)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what}
 
-    launches = args.steps * sum(kernels_per_forward(T, k, fp8) for T in Ts)
+    launches = args.steps * sum(kernels_per_forward(T, k, fp8, H) for T in Ts)
     if rank == 0:
         line = {"metric": "fused-MoE layer tokens/s", "value": value, "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

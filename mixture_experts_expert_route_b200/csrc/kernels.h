@@ -67,7 +67,13 @@ cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k,
                                        int capacity, int32_t* ids, float* w, int32_t* counts,
                                        int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
-                                       cudaStream_t s, int32_t* ctl = nullptr, int ctl_ints = 0);
+                                       cudaStream_t s, int32_t* ctl = nullptr, int ctl_ints = 0,
+                                       const void* x = nullptr, long x_elems = 0,
+                                       uint32_t* amax_out = nullptr);
+// Batches small enough for the single-CTA kernel to also take amax(x) (FP8):
+// up to 64 KB of x (measured on B200: at 184 KB the one CTA took longer than
+// the separate amax kernel it replaced).
+constexpr long kSmallAmaxElems = 32768;
 cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
                                  int capacity, int32_t* counts, int32_t* offsets,
                                  int32_t* sorted_ids, int32_t* inv_perm, int32_t* tiles,

@@ -96,6 +96,7 @@ struct FfnCall {
     void* y_perm;
     int32_t* status;
     int max_ctas;
+    bool x_amax_ready = false;   // amax(x) already in the control block (FP8)
 };
 
 void record(moe_event_t* ev, int i, cudaStream_t s) {
@@ -110,7 +111,8 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     uint32_t* amax_h = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxH);
     cudaError_t e;
     if (fp8) {
-        e = launch_amax_bf16(f.x, static_cast<long>(f.T) * f.H, amax_x, s);
+        e = f.x_amax_ready ? cudaSuccess
+                           : launch_amax_bf16(f.x, static_cast<long>(f.T) * f.H, amax_x, s);
         if (e == cudaSuccess)
             e = launch_gather_fp8(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, amax_x,
                                   f.w, b.x_perm, b.w_perm, s);
@@ -381,10 +383,15 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     // the status word when the caller gave none) once the previous call's
     // kernels are done with it.
     cudaError_t e;
-    if (fused_route_permute_ok(a->T, a->k)) {
-        e = launch_route_permute_small(a->logits, a->T, a->E, a->k, block_m, cap, ids, w, b.counts,
-                                       b.offsets, b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,
-                                       status, s, b.ffn.ctl, kCtlInts);
+    const long x_elems = static_cast<long>(a->T) * a->H;
+    const bool small = fused_route_permute_ok(a->T, a->k);
+    const bool amax_fused = small && a->dtype == MOE_FP8_E4M3 && x_elems <= kSmallAmaxElems;
+    if (small) {
+        e = launch_route_permute_small(
+            a->logits, a->T, a->E, a->k, block_m, cap, ids, w, b.counts, b.offsets, b.sorted_ids,
+            b.inv_perm, b.tiles, b.num_tiles, status, s, b.ffn.ctl, kCtlInts,
+            amax_fused ? a->x : nullptr, x_elems,
+            amax_fused ? reinterpret_cast<uint32_t*>(b.ffn.ctl + kCtlAmaxX) : nullptr);
     } else {
         e = launch_route_topk(a->logits, a->T, a->E, a->k, ids, w, s, b.ffn.ctl, kCtlInts);
         if (e == cudaSuccess)
@@ -395,7 +402,7 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 1, s);
     FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, cap, a->x, w, b.counts, b.offsets,
-              b.sorted_ids, a->packed, a->scales, b.y_perm, status, a->max_ctas};
+              b.sorted_ids, a->packed, a->scales, b.y_perm, status, a->max_ctas, amax_fused};
     st = run_ffn(f, b.ffn, ev, s);
     if (st != MOE_OK) return st;
     if (launch_combine(b.y_perm, b.inv_perm, a->T, a->k, a->H, a->out, s) != cudaSuccess)

@@ -37,6 +37,17 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kPermChunk = 512;
 constexpr int kScanBatch = 16;
 
+// Largest |value| of 8 packed bf16.
+__device__ __forceinline__ float amax8(uint4 v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(u[i] << 16)),
+                           fabsf(__uint_as_float(u[i] & 0xffff0000u))));
+    return m;
+}
+
 // Selection order as one 64-bit key, larger first: an order-preserving map of
 // the logit (-0 folded onto +0; NaN below every number) in the high word and
 // the complement of the expert index in the low word (equal logits: the lower
@@ -64,7 +75,8 @@ __device__ __forceinline__ float key_value(uint64_t key) {
 // summed per lane in ascending j and then across the warp.  ids and w are
 // written once at the end, lane j for entry j.
 template <int EPL>
-__device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w) {
+__device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w,
+                          int32_t* ids_copy = nullptr) {
     const int lane = threadIdx.x & 31;
     uint64_t key[EPL];
 #pragma unroll
@@ -91,18 +103,14 @@ __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w
         }
         const int bi = static_cast<int>(0xffffffffu - static_cast<uint32_t>(best));
         const float bv = key_value(best);
-        if ((bi & 31) == lane) {
+        // selects, not indexed stores, so the arrays stay in registers
+        const bool won = (bi & 31) == lane, keep = (j & 31) == lane;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == (bi >> 5)) key[i] = 0ull;
-        }
-        if ((j & 31) == lane) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == (j >> 5)) {
-                    sv[i] = bv;
-                    si[i] = bi;
-                }
+        for (int i = 0; i < EPL; ++i) {
+            key[i] = (won && i == (bi >> 5)) ? 0ull : key[i];
+            const bool here = keep && i == (j >> 5);
+            sv[i] = here ? bv : sv[i];
+            si[i] = here ? bi : si[i];
         }
         if (j == 0) m = bv;
     }
@@ -117,6 +125,7 @@ __device__ void warp_topk(const float* row, int E, int k, int32_t* ids, float* w
         const int j = lane + 32 * i;
         if (j < k) {
             ids[j] = si[i];
+            if (ids_copy) ids_copy[j] = si[i];
             w[j] = expf(sv[i] - m) / z;
         }
     }
@@ -253,11 +262,14 @@ __global__ void __launch_bounds__(kSmallThreads)
                                int capacity, int32_t* ids, float* w, int32_t* counts,
                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                int32_t* tiles, int32_t* num_tiles, int32_t* status, int32_t* ctl,
-                               int ctl_ints) {
+                               int ctl_ints, const uint4* __restrict__ x, long x_vecs,
+                               uint32_t* amax_out) {
     constexpr int NW = kSmallThreads / 32;
     __shared__ int hist[NW][kMaxExperts];
     __shared__ float slog[kStageFloats];
     __shared__ int tmp[NW + 1];
+    __shared__ int32_t sids[kChunk];   // the ids, read twice below
+    __shared__ float wmax[NW];
     const int warp = threadIdx.x >> 5;
     const long A = static_cast<long>(T) * k;
     pdl_wait();
@@ -273,12 +285,27 @@ __global__ void __launch_bounds__(kSmallThreads)
         }
         for (int t = warp; t < T; t += NW)
             warp_topk<EPL>(src + static_cast<long>(t) * E, E, k, ids + static_cast<long>(t) * k,
-                           w + static_cast<long>(t) * k);
+                           w + static_cast<long>(t) * k, sids + static_cast<long>(t) * k);
+    } else {
+        for (int i = threadIdx.x; i < A; i += kSmallThreads) sids[i] = ids[i];
     }
     for (int i = threadIdx.x; i < NW * kMaxExperts; i += kSmallThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    chunk_histogram<NW, kChunk>(ids, A, 0, E, hist, status);
+    // FP8 small batches: amax of x (a3's scale) here, saving a kernel; the
+    // control block was zeroed above, before the barrier
+    float xm = 0.0f;
+    if (amax_out) {
+        for (long i = threadIdx.x; i < x_vecs; i += kSmallThreads) xm = fmaxf(xm, amax8(x[i]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) xm = fmaxf(xm, __shfl_xor_sync(kFull, xm, off));
+        if ((threadIdx.x & 31) == 0) wmax[warp] = xm;
+    }
+    chunk_histogram<NW, kChunk>(sids, A, 0, E, hist, status);
     __syncthreads();
+    if (amax_out && threadIdx.x == 0) {
+        for (int i = 0; i < NW; ++i) xm = fmaxf(xm, wmax[i]);
+        *amax_out = __float_as_uint(xm);
+    }
     const int e = threadIdx.x;
     int c = 0;
     if (e < E)
@@ -296,7 +323,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     const int total = tmp[NW];
     __syncthreads();
     fill_tail<kSmallThreads>(total, block_m, capacity, sorted_ids, tiles);
-    chunk_scatter<NW, kChunk>(ids, A, 0, E, hist, sorted_ids, inv_perm);
+    chunk_scatter<NW, kChunk>(sids, A, 0, E, hist, sorted_ids, inv_perm);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -403,11 +430,14 @@ cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k,
                                        int capacity, int32_t* ids, float* w, int32_t* counts,
                                        int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
-                                       cudaStream_t s, int32_t* ctl, int ctl_ints) {
+                                       cudaStream_t s, int32_t* ctl, int ctl_ints, const void* x,
+                                       long x_elems, uint32_t* amax_out) {
+    const uint4* xv = static_cast<const uint4*>(x);
+    const long nv = x_elems / 8;
 #define MOE_SMALL(EPL)                                                                            \
     return launch_pdl(route_permute_small_kernel<EPL>, dim3(1), dim3(kSmallThreads), 0, s, logits, \
                       T, E, k, block_m, capacity, ids, w, counts, offsets, sorted_ids, inv_perm,  \
-                      tiles, num_tiles, status, ctl, ctl_ints)
+                      tiles, num_tiles, status, ctl, ctl_ints, xv, nv, amax_out)
     switch (epl_for(E)) {
         case 1: MOE_SMALL(1);
         case 2: MOE_SMALL(2);
