@@ -43,6 +43,28 @@ __global__ void __launch_bounds__(kThreads)
     for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
 }
 
+// Row/vector position of flat index i (row p, 16-byte vector v of a row of
+// vpr vectors), advanced through a grid-stride loop by additions only: the
+// per-element 64-bit division it replaces dominated the kernels' issue slots.
+struct RowVec {
+    int p, v, sq, sr, vpr;
+    __device__ __forceinline__ RowVec(long i0, long stride, int vpr_) : vpr(vpr_) {
+        p = static_cast<int>(i0 / vpr);
+        v = static_cast<int>(i0 - static_cast<long>(p) * vpr);
+        sq = static_cast<int>(stride / vpr);
+        sr = static_cast<int>(stride - static_cast<long>(sq) * vpr);
+    }
+    __device__ __forceinline__ void next() {
+        p += sq;
+        v += sr;
+        if (v >= vpr) {
+            v -= vpr;
+            ++p;
+        }
+    }
+    __device__ __forceinline__ long flat() const { return static_cast<long>(p) * vpr + v; }
+};
+
 // a3: X_perm[p] = x[sorted_ids[p] / k] for p < offsets[E]; pad rows are zero.
 // Also w_perm[p] = w[sorted_ids[p]] (0 for pads), the routing weight the down
 // GEMM's epilogue applies to row p.
@@ -54,15 +76,13 @@ __global__ void __launch_bounds__(kThreads)
     pdl_wait();
     pdl_trigger();
     const int rows = min(capacity, offsets[E]);
-    const long n = static_cast<long>(rows) * vec_per_row;
-    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < n;
-         i += static_cast<long>(gridDim.x) * kThreads) {
-        const int p = static_cast<int>(i / vec_per_row);
-        const int v = static_cast<int>(i - static_cast<long>(p) * vec_per_row);
-        const int sid = sorted_ids[p];
-        if (v == 0) w_perm[p] = sid >= 0 ? w[sid] : 0.0f;
-        x_perm[i] = sid >= 0 ? x[static_cast<long>(sid / k) * vec_per_row + v]
-                             : make_uint4(0, 0, 0, 0);
+    for (RowVec r(static_cast<long>(blockIdx.x) * kThreads + threadIdx.x,
+                  static_cast<long>(gridDim.x) * kThreads, vec_per_row);
+         r.p < rows; r.next()) {
+        const int sid = sorted_ids[r.p];
+        if (r.v == 0) w_perm[r.p] = sid >= 0 ? w[sid] : 0.0f;
+        x_perm[r.flat()] = sid >= 0 ? x[static_cast<long>(sid / k) * vec_per_row + r.v]
+                                    : make_uint4(0, 0, 0, 0);
     }
 }
 
@@ -97,14 +117,30 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-__device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+// Activations: e4m3 codes of 8 packed bf16 values times inv_s = 1/s (the
+// weights, quantised once, keep the correctly rounded x / s).  Scaling by the
+// reciprocal costs one multiply where an IEEE division took most of the
+// kernel's issue slots; a code can differ by one step from RNE(x / s) only
+// when x / s lies within an fp32 ulp of an e4m3 rounding midpoint.  Two
+// values per saturating RNE conversion.  A scale so small that 1/s overflows
+// (amax below ~1e-36) takes the division instead (0 * inf would be NaN).
+__device__ __forceinline__ uint2 quant8(uint4 v, float inv_s, float s) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[2] = {0, 0};
+    if (!(inv_s <= 3.0e38f)) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = fp8_quant(bf16_lo(w[i]), s);
+            const uint32_t hi = fp8_quant(bf16_hi(w[i]), s);
+            out[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+        }
+        return make_uint2(out[0], out[1]);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = fp8_quant(bf16_lo(w[i]), s);
-        const uint32_t hi = fp8_quant(bf16_hi(w[i]), s);
-        out[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+        const float2 f = make_float2(bf16_lo(w[i]) * inv_s, bf16_hi(w[i]) * inv_s);
+        const uint32_t pair = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        out[i >> 1] |= pair << (16 * (i & 1));
     }
     return make_uint2(out[0], out[1]);
 }
@@ -119,16 +155,15 @@ __global__ void __launch_bounds__(kThreads)
     pdl_wait();
     pdl_trigger();
     const int rows = min(capacity, offsets[E]);
-    const long n = static_cast<long>(rows) * vec_per_row;
     const float s = fp8_scale_from_amax(*amax_bits);
-    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < n;
-         i += static_cast<long>(gridDim.x) * kThreads) {
-        const int p = static_cast<int>(i / vec_per_row);
-        const int v = static_cast<int>(i - static_cast<long>(p) * vec_per_row);
-        const int sid = sorted_ids[p];
-        if (v == 0) w_perm[p] = sid >= 0 ? w[sid] : 0.0f;
-        x_perm[i] = sid >= 0 ? quant8(x[static_cast<long>(sid / k) * vec_per_row + v], s)
-                             : make_uint2(0, 0);
+    const float inv_s = 1.0f / s;
+    for (RowVec r(static_cast<long>(blockIdx.x) * kThreads + threadIdx.x,
+                  static_cast<long>(gridDim.x) * kThreads, vec_per_row);
+         r.p < rows; r.next()) {
+        const int sid = sorted_ids[r.p];
+        if (r.v == 0) w_perm[r.p] = sid >= 0 ? w[sid] : 0.0f;
+        x_perm[r.flat()] = sid >= 0 ? quant8(x[static_cast<long>(sid / k) * vec_per_row + r.v], inv_s, s)
+                                    : make_uint2(0, 0);
     }
 }
 
@@ -142,9 +177,10 @@ __global__ void __launch_bounds__(kThreads)
     const int rows = min(capacity, offsets[E]);
     const long n = static_cast<long>(rows) * vec_per_row;
     const float s = fp8_scale_from_amax(*amax_bits);
+    const float inv_s = 1.0f / s;
     for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < n;
          i += static_cast<long>(gridDim.x) * kThreads)
-        dst[i] = quant8(src[i], s);
+        dst[i] = quant8(src[i], inv_s, s);
 }
 
 // a7: out[t] = sum_j y_perm[inv_perm[t*k + j]] in fp32, j ascending.
@@ -155,7 +191,10 @@ __global__ void __launch_bounds__(kThreads)
     pdl_trigger();
     const long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x;
     if (i >= static_cast<long>(T) * vec_per_row) return;
-    const long t = i / vec_per_row;
+    // 32-bit division whenever the index fits (a 64-bit one is ~5x the work)
+    const long t = (i >> 32) == 0 ? static_cast<long>(static_cast<uint32_t>(i) /
+                                                     static_cast<uint32_t>(vec_per_row))
+                                  : i / vec_per_row;
     const int v = static_cast<int>(i - t * vec_per_row);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
