@@ -24,18 +24,24 @@
 // Roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (single
 // thread), warp 2 = TMEM allocator, warps 4-11 = epilogue (two warps per
 // 32-lane TMEM quarter, alternating 16-column chunks).
-// smem ring of 2 stages of kps k-blocks (A kps*16 KB + B kps*nmax*128 B),
-// 128-byte swizzle; two TMEM
-// accumulators of nmax fp32 columns so the epilogue of one unit overlaps the
+// Shared-memory ring of stages of KPS k-blocks (A KPS*16 KB + B KPS*rows*128 B,
+// 128-byte swizzle): 2 stages of 4 k-blocks on one CTA (token tiles of at most
+// 64 rows), 3 stages of 2 k-blocks per CTA of a pair (larger tiles).  Two TMEM
+// accumulators of nmax fp32 columns let the epilogue of one unit overlap the
 // main loop of the next.  Every wait is bounded; on expiry the kernel records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 //
+// Token tiles of more than 64 rows run on CTA pairs (cta_group::2): M = 256
+// weight rows per MMA, each CTA holding 128 of them and half of the token
+// tile; the rank-0 CTA issues the MMAs and its barriers count both CTAs' copies.
+//
 // Weights (A) are pre-packed as 16 KB tiles that are already the swizzled
 // shared-memory image of one stage, so a stage's A operand (one to four
-// consecutive k-blocks) is one contiguous bulk copy.  Activations (B) come through TMA tensor maps with 64-row
-// and 16-row boxes, so a token tile moves only its own rows.  Launched with
-// programmatic dependent launch: the producer fetches the first weight tiles
-// before waiting for the previous kernel, whose output (B) it loads after.
+// consecutive k-blocks) is one contiguous copy.  Activations (B) come through
+// TMA tensor maps with 128-, 64- and 16-row boxes, so a token tile moves only
+// its own rows.  Launched with programmatic dependent launch: the producer
+// fetches the first weight tiles before waiting for the previous kernel, whose
+// output (B) it loads after.
 #include <cstring>
 #include <mutex>
 

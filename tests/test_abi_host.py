@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import oracle
 
@@ -122,3 +123,15 @@ def test_forward_argument_errors(L):
     assert call(_fwd(L), 64) == WS                            # workspace too small
     assert call(_fwd(L, T=0, x=None, logits=None)) == 0       # T = 0 no-op
     assert lib.moe_forward(None, ws, big, None) == INVALID
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No silent fallback: without the built library the binding raises."""
+    import mixture_experts_expert_route_b200._lib as binding
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(ImportError):
+        binding.lib()
+    # and a CUDA tensor argument is required: host tensors are refused, not copied
+    with pytest.raises(ValueError):
+        binding._ptr(torch.zeros(1))
