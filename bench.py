@@ -44,7 +44,8 @@ NBATCH = 4
 GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
 # DRAM bytes (read + write) of one gate/up launch from an ncu capture of the
 # same kernel build, keyed by (workload, T); None until captured.
-TRAFFIC = {("decode", 64): 1887167120, ("prefill", 4096): 1378159440}
+TRAFFIC = {("decode", 64): 1887167120, ("prefill", 4096): 1378159440,
+           ("fp8", 2048): 876559360}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
 
