@@ -19,6 +19,7 @@ collective), timed on the device and reduced as the max over ranks.
 from __future__ import annotations
 
 import argparse
+import atexit
 import json
 import os
 import statistics
@@ -74,7 +75,10 @@ def kernels_per_forward(T, k, fp8, H):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled every 25 ms; the summary
+    keeps the samples that arrived between mark_start() and mark_end() (the
+    timed regions), or all of them, flagged, when none did."""
+    INTERVAL_MS = 25
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
@@ -83,23 +87,30 @@ class ClockSampler:
         u = str(uuid)
         self.uuid = u if u.startswith("GPU-") else "GPU-" + u
         self.proc, self.lines, self.err = None, [], ""
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             threading.Thread(target=self._read, daemon=True).start()
             threading.Thread(target=self._read_err, daemon=True).start()
-            time.sleep(0.3)   # first sample before the timed region starts
+            time.sleep(0.3)   # the first samples arrive before the timed region starts
         except (OSError, ValueError) as e:
             self.proc, self.err = None, str(e)
         return self
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            self.lines.append((time.perf_counter(), ln.strip()))
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def _read_err(self):
         for ln in self.proc.stderr:
@@ -116,7 +127,17 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        window = "timed regions"
+        if self.t0 is not None and self.t1 is not None:
+            # a sample printed up to one interval after the region ends was taken inside it
+            late = 2 * self.INTERVAL_MS / 1e3
+            inside = [(t, ln) for t, ln in lines if self.t0 <= t <= self.t1 + late]
+            if inside:
+                lines = inside
+            else:
+                window = "no sample inside the timed regions; all samples"
+        for _, ln in lines:
             f = [v.strip() for v in ln.split(",")]
             if len(f) < 7:
                 continue
@@ -129,7 +150,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-               "reasons": sorted(reasons), "samples": len(sm)}
+               "reasons": sorted(reasons), "samples": len(sm), "window": window}
         if not sm:
             out["error"] = (self.err.strip() or "no samples")[:200]
         return out
@@ -310,12 +331,14 @@ def run_native(args):
     torch.cuda.synchronize()
     # headline region: the layer exactly as a caller runs it (no stage events,
     # so consecutive kernels keep their programmatic-launch overlap)
-    with ClockSampler(uuid) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t_end.record(stream)
-        torch.cuda.synchronize()
+    clk = ClockSampler(uuid).__enter__()
+    atexit.register(clk.__exit__, None, None, None)   # stop the sampler on any exit path
+    clk.mark_start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t_end.record(stream)
+    torch.cuda.synchronize()
     if dist:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
@@ -334,6 +357,8 @@ def run_native(args):
     for i in range(args.steps):
         step(i, evs[i])
     torch.cuda.synchronize()
+    clk.mark_end()     # the headline and stage regions, back to back
+    clk.__exit__(None, None, None)
 
     # per-stage device times from the events recorded inside the timed region
     stage = {T: [[] for _ in range(6)] for T in Ts}
