@@ -108,11 +108,12 @@ class Weights:
 
 def make_weights(name: str, seed: int = 0, device: str = "cpu", E: int | None = None,
                  k: int | None = None, H: int | None = None, I: int | None = None,
-                 zero_router: bool = False) -> Weights:
+                 zero_router: bool = False, router_only: bool = False) -> Weights:
     """Router and expert weights of a workload.  Generator(seed) draws, in order,
     W_r, the Zipf ranks (skewed only), then W_g, W_u, W_d one expert at a time.
     On a CUDA ``device`` the expert weights come from a CUDA generator seeded
-    seed + 1 (different values, same distribution)."""
+    seed + 1 (different values, same distribution).  ``router_only`` stops after
+    the router (same W_r and bias; the expert tensors are left empty)."""
     cfg = dict(CONFIGS[name])
     H = H or cfg["H"]
     I = I or cfg["I"]
@@ -124,6 +125,9 @@ def make_weights(name: str, seed: int = 0, device: str = "cpu", E: int | None = 
     if zero_router:
         Wr.zero_()
     bias = zipf_bias(E, gen) if cfg.get("zipf") else torch.zeros(E, dtype=torch.float32)
+    if router_only:
+        empty = torch.empty(0, dtype=wdtype)
+        return Weights(name, H, I, E, k, empty, empty, empty, Wr, bias)
     wgen = gen if device == "cpu" else torch.Generator(device=device).manual_seed(seed + 1)
     Wg = torch.empty((E, H, I), dtype=wdtype, device=device)
     Wu = torch.empty((E, H, I), dtype=wdtype, device=device)
