@@ -167,6 +167,9 @@ MOE_API moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const 
  *                                           then quantised with s_h)
  *   y_perm[p] = w[sorted_ids[p]] * (h[p] W_d[e])   (bf16; 0 for pads)
  * for every row p of expert e's block.  Inputs come from moe_align_permute.
+ * FP8 activations are coded as RNE_sat(v * (1/s)) with the fp32 reciprocal of
+ * their scale (a code may differ by one step from RNE(v / s) when v / s lies
+ * within an fp32 ulp of a rounding midpoint); weights use v / s exactly.
  * max_ctas > 0 caps the persistent grid (0 = one CTA per SM).
  * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE
  * synchronously; device faults in *status (or, if status is NULL, in the
