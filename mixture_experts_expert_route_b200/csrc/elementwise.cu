@@ -1,7 +1,8 @@
 // elementwise.cu -- the layer's memory-bound steps: a3 gather (+ FP8
 // quantisation of x), a5 FP8 quantisation of h, a7 combine, the one-time
 // weight packing, and the failure-detection self-test.  All are HBM-bound:
-// 16-byte vector accesses, one warp per row, grids sized from the data.
+// 16-byte vector accesses, one vector per thread (one warp per row for large
+// bf16 gathers), grids sized from the data.
 #include "common.cuh"
 #include "kernels.h"
 
