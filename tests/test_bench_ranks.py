@@ -57,3 +57,24 @@ def test_reference_arm_other_ranks_exit_quietly():
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_bench_mirrors_library_dispatch_constants():
+    """bench.py counts the kernels a forward launches from the library's
+    dispatch limits; its copies of those limits must match kernels.h."""
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+    src = open(os.path.join(ROOT, "mixture_experts_expert_route_b200", "csrc",
+                            "kernels.h")).read()
+    def const(name):
+        return int(re.search(rf"constexpr\s+\w+\s+{name}\s*=\s*(\d+)", src).group(1))
+    assert bench.SMALL_T == const("kSmallT")
+    assert bench.CHUNK == const("kChunk")
+    assert bench.SMALL_AMAX == const("kSmallAmaxElems")
+    # decode T=1 (small path, bf16): route+permute, gather, gate/up, down, combine
+    assert bench.kernels_per_forward(1, 2, False, 4096) == 5
+    # FP8 T=1, x of 5.6 KB: amax folded into the route kernel, plus h quantisation
+    assert bench.kernels_per_forward(1, 4, True, 2880) == 6
+    # FP8 T=2048: route, 3 permutation kernels, amax, gather, 2 GEMMs, quant, combine
+    assert bench.kernels_per_forward(2048, 4, True, 2880) == 10
