@@ -204,6 +204,12 @@ def oracle_sample(W, dtype, Ts, budget_s=12.0):
     return n / el, oracle.num_threads(), what
 
 
+def weight_device(name):
+    """Where a workload's expert weights are drawn: the skewed workload's on the
+    GPU (22.5 GB), the others on the CPU; both arms use the same rule."""
+    return "cuda" if name == "skewed" and torch.cuda.is_available() else "cpu"
+
+
 def aggregate_over_ranks(elapsed_ms, tokens_per_step, steps, world, dist=None, device=None):
     """Whole-job throughput of a timed region: the slowest rank's time (max over
     ranks) and the tokens all ranks processed in it.  Returns (ms, tokens/s)."""
@@ -219,7 +225,10 @@ def run_reference(args):
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
-    W = make_weights(wl["cfg"], 0, "cpu")
+    # the same weights as the native arm (the skewed workload's 22.5 GB of
+    # expert weights are drawn on the GPU there; the oracle copies the experts
+    # its sample uses to the host)
+    W = make_weights(wl["cfg"], 0, weight_device(wl["cfg"]))
     Ts = CONFIGS[wl["cfg"]]["T"]
     budget = args.ref_step_seconds
     for _ in range(args.warmup):
@@ -262,7 +271,7 @@ def run_native(args):
     cfg = CONFIGS[name]
     Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else cfg["T"]
     k, E, H, I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
-    W = make_weights(name, 0, "cuda" if name == "skewed" else "cpu")
+    W = make_weights(name, 0, weight_device(name))
     Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (W.Wg, W.Wu, W.Wd))
     layer = moe.MoELayer(Wg, Wu, Wd, k=k, dtype=dtype)
     del Wg, Wu, Wd
