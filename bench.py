@@ -1,27 +1,35 @@
 #!/usr/bin/env python
 """Benchmark of the fused MoE layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all]
                     [--impl native|reference]
 
 A step is one pass of the whole layer (route -> permute -> gather -> gate/up
-GEMM -> [FP8 h quant] -> down GEMM -> combine) over one batch of every token
-count of the workload, e.g. T = 1, 4, 16, 64 for the decode workload
-(H=4096, I=14336, E=8, top-2, bf16).  Inputs are seeded synthetic tensors;
-the expert weights (2.8 GB for decode) are larger than the 126 MB L2 and
-four input batches rotate between steps.
+GEMM -> [FP8 h quant] -> down GEMM -> combine) over one
+batch of every token count of a workload, e.g. T = 1, 4, 16, 64 for the
+decode workload (H=4096, I=14336, E=8, top-2, bf16).  Inputs are seeded
+synthetic tensors; the expert weights are larger than the 126 MB L2 and four
+input batches rotate between steps.
+
+With the default ``--workload all`` the headline (``value``, ``roofline``,
+``e2e``, ``cpu_baseline``) is the decode workload, and the same JSON line
+carries a ``workloads`` block with the other workloads measured the same way
+on the same GPU: fine-grained prefill (T=4096), FP8 (T = 1, 32, 256, 2048) and
+the skewed large-expert-count layer (T=8192).
 
 Metric: layer tokens/s (whole job, all ranks).  N > 1 runs independent
 replicas, one per GPU (the layer is single-GPU; there is no data-path
 collective), timed on the device and reduced as the max over ranks.
-`--impl reference` times the CPU oracle on a bounded sample instead.
+``--impl reference`` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
 
 import argparse
 import atexit
+import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -41,14 +49,36 @@ WORKLOADS = {
     "fp8": dict(cfg="fp8", dtype=1, bound="tensor"),      # roofline entry at T=2048
     "skewed": dict(cfg="skewed", dtype=0, bound="tensor"),
 }
+HEADLINE = "decode"
 NBATCH = 4
 GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
-# DRAM bytes (read + write) of one gate/up launch from an ncu capture of the
-# same kernel build, keyed by (workload, T); None until captured.
-TRAFFIC = {("decode", 64): 1887167120, ("prefill", 4096): 1378159440,
-           ("fp8", 2048): 876559360}
+# DRAM bytes (read + write) of one gate/up launch, from an ncu capture made
+# offline (profiles/), keyed by (workload, T).  Each value records the hash of
+# the GEMM's source files it was captured with; the bench reports it only
+# while the sources still hash the same, and null (stale) otherwise.
+GEMM_SOURCES = ("mixture_experts_expert_route_b200/csrc/grouped_gemm.cu",
+                "mixture_experts_expert_route_b200/csrc/common.cuh")
+TRAFFIC = {}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_for(workload, T):
+    """(bytes or None, note) for the roofline's `traffic` field."""
+    rec = TRAFFIC.get((workload, T))
+    if rec is None:
+        return None, "no ncu capture of this build"
+    if rec["gemm_src"] != gemm_source_hash():
+        return None, f"stale: captured on GEMM sources {rec['gemm_src']} ({rec['capture']})"
+    return rec["bytes"], f"ncu capture offline ({rec['capture']}), GEMM sources {rec['gemm_src']}"
 
 
 def describe(name):
@@ -167,41 +197,83 @@ def peaks():
 
 def gate_up_bytes(T, k, H, I, active, fp8):
     """Algorithmic bytes of one gate/up launch: the active experts' W_g and W_u,
-    the T*k gathered activation rows read, the T*k rows of h written (bf16)."""
+    the T tokens' activation rows read (each once), the T*k rows of h written."""
     wb = 1 if fp8 else 2
-    return active * 2 * H * I * wb + T * k * H * wb + T * k * I * 2
+    return active * 2 * H * I * wb + T * H * wb + T * k * I * 2
 
 
-def oracle_sample(W, dtype, Ts, budget_s=12.0):
-    """The oracle on a bounded sample: tokens of the largest batch, one by one,
-    until the time budget is spent.  Returns (tokens/s, cores, description)."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(W, dtype, T, budget_s=12.0, max_tokens=None, threads=None):
+    """The oracle on a bounded sample: tokens of batch 0 with T tokens, one
+    call per `threads` tokens, until the time budget is spent.  Only the
+    experts the first `max_tokens` tokens use are copied to the host.  The
+    FP8 oracle needs every h row for its scale, so it runs whole batches.
+    Returns (tokens/s, threads used, description)."""
     import numpy as np
     import oracle
-    T = max(Ts)
     x, logits = make_batch(W, T, 0, 0)
+    n_pool = T if max_tokens is None else min(T, max_tokens)
+    x, logits = x[:n_pool], logits[:n_pool]
     ids, w = oracle.route_topk(logits, W.k)
     used = sorted(set(int(e) for e in np.unique(ids)))
-    remap = {e: i for i, e in enumerate(used)}
+    remap = np.zeros(W.E, np.int32)
+    remap[used] = np.arange(len(used), dtype=np.int32)
     Wg = W.Wg[used].cpu().to(torch.bfloat16)
     Wu = W.Wu[used].cpu().to(torch.bfloat16)
     Wd = W.Wd[used].cpu().to(torch.bfloat16)
-    lid = np.vectorize(remap.get)(ids).astype(np.int32)
-    n, t0 = 0, time.perf_counter()
-    step = max(1, oracle.num_threads())
-    while True:
-        toks = [(n + i) % T for i in range(step)]
-        if dtype == 0:
-            oracle.moe_layer(x, lid, w, Wg, Wu, Wd, tokens=toks)
-        else:   # the FP8 oracle needs every h row for its scale: whole batch
-            oracle.moe_layer_fp8(x, lid, w, Wg, Wu, Wd, tokens=toks)
-            n += T - step
-        n += step
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    el = time.perf_counter() - t0
-    what = (f"oracle layer on {n} tokens of the T={T} batch ({budget_s:.0f} s budget), "
-            f"{len(used)} experts")
-    return n / el, oracle.num_threads(), what
+    lid = remap[ids]
+    saved = oracle.num_threads()
+    if threads is not None:
+        oracle.set_num_threads(threads)
+    used_threads = oracle.num_threads()
+    try:
+        n, t0 = 0, time.perf_counter()
+        step = max(1, used_threads)
+        while True:
+            if dtype == 0:
+                toks = [(n + i) % n_pool for i in range(step)]
+                oracle.moe_layer(x, lid, w, Wg, Wu, Wd, tokens=toks)
+                n += step
+            else:
+                oracle.moe_layer_fp8(x, lid, w, Wg, Wu, Wd)
+                n += n_pool
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        el = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(saved)
+    what = (f"oracle layer on {n} tokens from the first {n_pool} of the T={T} batch "
+            f"({budget_s:.0f} s budget), {len(used)} experts, {used_threads} threads")
+    return n / el, used_threads, what
+
+
+def cpu_baseline(W, dtype, T, budget_s, max_tokens=None, single_thread=True):
+    v, cores, what = oracle_sample(W, dtype, T, budget_s, max_tokens)
+    out = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what,
+           "cpu_model": cpu_model()}
+    if single_thread:
+        v1, _, what1 = oracle_sample(W, dtype, T, budget_s, max_tokens, threads=1)
+        out["single_thread_value"] = v1
+        out["single_thread_sample"] = what1
+    return out
+
+
+# oracle sample per workload: (T of the batch it draws tokens from, the
+# token pool: only the first tokens, whose experts are copied to the host;
+# None = the whole batch).  The FP8 oracle runs whole batches (its h scale
+# needs every row), hence its small batch.
+ORACLE_SAMPLE = {"decode": (64, None), "prefill": (4096, 512), "fp8": (32, None),
+                 "skewed": (8192, 32)}
 
 
 def weight_device(name):
@@ -220,23 +292,28 @@ def aggregate_over_ranks(elapsed_ms, tokens_per_step, steps, world, dist=None, d
     return ms, tokens_per_step * steps * world / (ms / 1e3)
 
 
+def headline_name(args):
+    return HEADLINE if args.workload == "all" else args.workload
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    name = headline_name(args)
+    wl = WORKLOADS[name]
     # the same weights as the native arm (the skewed workload's 22.5 GB of
     # expert weights are drawn on the GPU there; the oracle copies the experts
     # its sample uses to the host)
     W = make_weights(wl["cfg"], 0, weight_device(wl["cfg"]))
-    Ts = CONFIGS[wl["cfg"]]["T"]
+    T, pool = ORACLE_SAMPLE[name]
     budget = args.ref_step_seconds
     for _ in range(args.warmup):
-        oracle_sample(W, wl["dtype"], Ts, budget_s=min(1.0, budget))
+        oracle_sample(W, wl["dtype"], T, budget_s=min(1.0, budget), max_tokens=pool)
     vals, cores, what = [], 1, ""
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        v, cores, what = oracle_sample(W, wl["dtype"], Ts, budget_s=budget)
+        v, cores, what = oracle_sample(W, wl["dtype"], T, budget_s=budget, max_tokens=pool)
         vals.append(v)
     el = time.perf_counter() - t0
     value = statistics.mean(vals)
@@ -245,222 +322,241 @@ def run_reference(args):
             "ms_per_step": 1e3 * el / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": describe(args.workload)},
+            "config": {"workload": describe(name)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle", "sample": what},
+                             "kind": "oracle", "sample": what, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_native(args):
-    import mixture_experts_expert_route_b200 as moe
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    wl = WORKLOADS[args.workload]
-    name, dtype = wl["cfg"], wl["dtype"]
-    cfg = CONFIGS[name]
-    Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else cfg["T"]
-    k, E, H, I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
-    W = make_weights(name, 0, weight_device(name))
-    Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (W.Wg, W.Wu, W.Wd))
-    layer = moe.MoELayer(Wg, Wu, Wd, k=k, dtype=dtype)
-    del Wg, Wu, Wd
-    batches = {T: [make_batch(W, T, 0, b) for b in range(NBATCH)] for T in Ts}
-    dev_in = {T: [(x.to(dev), lg.to(dev)) for x, lg in batches[T]] for T in Ts}
-    outs = {T: torch.empty((T, H), dtype=torch.bfloat16, device=dev) for T in Ts}
-    for T in Ts:
-        layer.workspace(T)
-    stream = torch.cuda.current_stream()
+class Bench:
+    """One workload on this rank's GPU: packed layer, rotating input batches,
+    the timed regions and the derived roofline figures."""
 
-    # active experts of every batch (for the algorithmic bytes)
-    active = {}
-    for T in Ts:
-        active[T] = []
-        for x, lg in dev_in[T]:
-            ids, _ = moe.route_topk(lg, k)
-            active[T].append(int(torch.unique(ids).numel()))
+    def __init__(self, name, args, dev, dist, world, Ts=None):
+        import mixture_experts_expert_route_b200 as moe
+        self.moe, self.name, self.args, self.dev, self.dist, self.world = \
+            moe, name, args, dev, dist, world
+        wl = WORKLOADS[name]
+        self.dtype = wl["dtype"]
+        self.fp8 = self.dtype == 1
+        cfg = CONFIGS[wl["cfg"]]
+        self.Ts = Ts or cfg["T"]
+        self.k, self.E, self.H, self.I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
+        self.W = make_weights(wl["cfg"], 0, weight_device(wl["cfg"]))
+        Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (self.W.Wg, self.W.Wu, self.W.Wd))
+        self.layer = moe.MoELayer(Wg, Wu, Wd, k=self.k, dtype=self.dtype)
+        del Wg, Wu, Wd
+        self.batches = {T: [make_batch(self.W, T, 0, b) for b in range(NBATCH)]
+                        for T in self.Ts}
+        self.dev_in = {T: [(x.to(dev), lg.to(dev)) for x, lg in self.batches[T]]
+                       for T in self.Ts}
+        self.outs = {T: torch.empty((T, self.H), dtype=torch.bfloat16, device=dev)
+                     for T in self.Ts}
+        for T in self.Ts:
+            self.layer.workspace(T)
+        self.stream = torch.cuda.current_stream()
+        self.active = {}
+        for T in self.Ts:
+            self.active[T] = []
+            for x, lg in self.dev_in[T]:
+                ids, _ = moe.route_topk(lg, self.k)
+                self.active[T].append(int(torch.unique(ids).numel()))
+        self.graphs, self.graph_note = {}, None
 
-    # Small token counts (T <= 64) run as CUDA graphs, one per rotating batch:
-    # there the layer is a short chain of short kernels and the launch cost
-    # on the host would otherwise show.  Larger T launch directly.
-    graphs, graph_note = {}, None
+    def release(self):
+        for gl in self.graphs.values():
+            for g in gl:
+                g.reset()
+        self.graphs.clear()
+        del self.layer, self.dev_in, self.outs, self.batches
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
 
-    def step(i, ev=None, direct=False):
-        for T in Ts:
-            if T in graphs and ev is None and not direct:
-                graphs[T][i % NBATCH].replay()
+    def check(self):
+        if self.layer.check() != 0:
+            raise RuntimeError(f"{self.name}: device status word reports a fault")
+
+    def step(self, i, ev=None, direct=False):
+        for T in self.Ts:
+            if T in self.graphs and ev is None and not direct:
+                self.graphs[T][i % NBATCH].replay()
                 continue
-            x, lg = dev_in[T][i % NBATCH]
-            layer(x, lg, out=outs[T], events=None if ev is None else ev[T])
+            x, lg = self.dev_in[T][i % NBATCH]
+            self.layer(x, lg, out=self.outs[T], events=None if ev is None else ev[T])
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    if layer.check() != 0:
-        raise RuntimeError("device status word reports a fault")
-    if not args.no_graphs:
+    def capture_graphs(self):
+        """Small token counts (T <= 64) run as CUDA graphs, one per rotating
+        batch: there the layer is a short chain of short kernels and the launch
+        cost on the host would otherwise show.  Larger T launch directly."""
+        if self.args.no_graphs:
+            return
         try:
-            for T in Ts:
+            for T in self.Ts:
                 if T > GRAPH_MAX_T:
                     continue
                 gl = []
                 for b in range(NBATCH):
-                    x, lg = dev_in[T][b]
+                    x, lg = self.dev_in[T][b]
                     g = torch.cuda.CUDAGraph()
                     with torch.cuda.graph(g):
-                        layer(x, lg, out=outs[T])
+                        self.layer(x, lg, out=self.outs[T])
                     gl.append(g)
-                graphs[T] = gl
-            for i in range(args.warmup):
-                step(i)
+                self.graphs[T] = gl
+            for i in range(self.args.warmup):
+                self.step(i)
             torch.cuda.synchronize()
-            if layer.check() != 0:
-                raise RuntimeError("device status word reports a fault")
+            self.check()
         except RuntimeError as ex:
             if "status word" in str(ex):
                 raise
-            graphs.clear()
-            graph_note = "graph capture failed, direct launches: " + str(ex).splitlines()[0]
+            self.graphs.clear()
+            self.graph_note = "graph capture failed, direct launches: " + str(ex).splitlines()[0]
 
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    uuid = torch.cuda.get_device_properties(dev).uuid
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    # headline region: the layer exactly as a caller runs it (no stage events,
-    # so consecutive kernels keep their programmatic-launch overlap)
-    clk = ClockSampler(uuid).__enter__()
-    atexit.register(clk.__exit__, None, None, None)   # stop the sampler on any exit path
-    clk.mark_start()
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(i)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if layer.check() != 0:
-        raise RuntimeError("device status word reports a fault")
-    tokens_per_step = sum(Ts)
-    elapsed_ms, value = aggregate_over_ranks(elapsed_ms, tokens_per_step, args.steps, world,
-                                             dist if world > 1 else None, dev)
+    def measure(self, clk):
+        """Headline region (the layer as a caller runs it), stage region
+        (events between the stages) and per-T regions.  Returns a result dict."""
+        args, dist, world = self.args, self.dist, self.world
+        for i in range(args.warmup):
+            self.step(i)
+        torch.cuda.synchronize()
+        self.check()
+        self.capture_graphs()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()     # the clock window: headline, stage and per-T regions
+        t_start.record(self.stream)
+        for i in range(args.steps):
+            self.step(i)
+        t_end.record(self.stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        elapsed_ms = t_start.elapsed_time(t_end)
+        self.check()
+        tokens_per_step = sum(self.Ts)
+        elapsed_ms, value = aggregate_over_ranks(elapsed_ms, tokens_per_step, args.steps, world,
+                                                 dist, self.dev)
 
-    # stage region: the same steps with CUDA events recorded between the
-    # layer's stages on the launching stream (an event between two kernels
-    # ends their overlap, so stage times are slightly pessimistic)
-    evs = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(7)] for T in Ts}
-           for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
-    clk.mark_end()     # the headline and stage regions, back to back
-    clk.__exit__(None, None, None)
+        # stage region: the same steps with CUDA events recorded between the
+        # layer's stages on the launching stream (an event between two kernels
+        # ends their overlap, so stage times are slightly pessimistic)
+        evs = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(7)] for T in self.Ts}
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            self.step(i, evs[i])
+        torch.cuda.synchronize()
+        stage = {T: [[] for _ in range(6)] for T in self.Ts}
+        for i in range(args.steps):
+            for T in self.Ts:
+                e = evs[i][T]
+                for s in range(6):
+                    stage[T][s].append(e[s].elapsed_time(e[s + 1]))
+        gu_ms = {T: statistics.mean(stage[T][2]) for T in self.Ts}
+        dn_ms = {T: statistics.mean(stage[T][4]) for T in self.Ts}
+        layer_ms = {T: statistics.mean([sum(stage[T][s][j] for s in range(6))
+                                        for j in range(args.steps)]) for T in self.Ts}
+        # whole-layer time of each T on its own (graph replays where the
+        # headline uses them; the direct-launch time is reported beside it)
+        layer_graph_ms = {}
+        for T in self.graphs:
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for i in range(args.steps):
+                self.graphs[T][i % NBATCH].replay()
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            layer_graph_ms[T] = e0.elapsed_time(e1) / args.steps
+        layer_direct_ms = {}
+        for T in self.Ts:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            x, lg = self.dev_in[T][0]
+            self.layer(x, lg, out=self.outs[T])
+            torch.cuda.synchronize()
+            e0.record(self.stream)
+            for i in range(args.steps):
+                x, lg = self.dev_in[T][i % NBATCH]
+                self.layer(x, lg, out=self.outs[T])
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            layer_direct_ms[T] = e0.elapsed_time(e1) / args.steps
+        clk.mark_end()
+        self.check()
+        return dict(elapsed_ms=elapsed_ms, value=value, gu_ms=gu_ms, dn_ms=dn_ms,
+                    layer_ms=layer_ms, layer_graph_ms=layer_graph_ms,
+                    layer_direct_ms=layer_direct_ms)
 
-    # per-stage device times from the events recorded inside the timed region
-    stage = {T: [[] for _ in range(6)] for T in Ts}
-    for i in range(args.steps):
+    def report(self, r):
+        """roofline + per-T figures of a measure() result."""
+        k, E, H, I, fp8, Ts = self.k, self.E, self.H, self.I, self.fp8, self.Ts
+        hbm, tf, src = peaks()
+        tpeak = tf * (2 if fp8 else 1)   # e4m3 dense peak = 2x the measured bf16 peak (nominal)
+        gu_ms = r["gu_ms"]
+        gu_bytes = {T: statistics.mean(gate_up_bytes(T, k, H, I, a, fp8)
+                                       for a in self.active[T]) for T in Ts}
+        gu_flops = {T: 4.0 * T * k * H * I for T in Ts}   # 2 GEMMs of 2*H*I per assignment
+        Tr = max(Ts)
+        kname = "grouped_gemm_kernel<%s, gate/up> at T=%d" % ("e4m3" if fp8 else "bf16", Tr)
+        traffic, tnote = traffic_for(self.name, Tr)
+        if WORKLOADS[self.name]["bound"] == "hbm":
+            achieved = gu_bytes[Tr] / (gu_ms[Tr] / 1e3) / 1e9
+            agg = sum(gu_bytes[T] for T in Ts) / (sum(gu_ms[T] for T in Ts) / 1e3) / 1e9
+            roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
+                        "traffic_note": tnote, "kernel": kname,
+                        "bytes_per_launch": int(gu_bytes[Tr]),
+                        "all_T_achieved": round(agg, 1), "all_T_frac": round(agg / hbm, 4),
+                        "peak_source": src + " (HBM copy)"}
+        else:
+            achieved = gu_flops[Tr] / (gu_ms[Tr] / 1e3) / 1e12
+            roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak,
+                        "unit": "TFLOP/s", "frac": round(achieved / tpeak, 4),
+                        "traffic": traffic, "traffic_note": tnote, "kernel": kname,
+                        "flops_per_launch": int(gu_flops[Tr]),
+                        "peak_source": src + (" (bf16 burst x2 for e4m3)" if fp8
+                                              else " (bf16 burst)")}
+        wb = 1 if fp8 else 2
+        per_T = {}
         for T in Ts:
-            e = evs[i][T]
-            for s in range(6):
-                stage[T][s].append(e[s].elapsed_time(e[s + 1]))
-    gu_ms = {T: statistics.mean(stage[T][2]) for T in Ts}
-    dn_ms = {T: statistics.mean(stage[T][4]) for T in Ts}
-    layer_ms = {T: statistics.mean([sum(stage[T][s][j] for s in range(6))
-                                    for j in range(args.steps)]) for T in Ts}
-    # whole-layer time of each T inside the headline region, from a third pass
-    # of single-T steps timed without stage events (graph replays where the
-    # headline uses them; the direct-launch time is reported beside it)
-    layer_graph_ms = {}
-    for T in graphs:
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs[T][i % NBATCH].replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        layer_graph_ms[T] = e0.elapsed_time(e1) / args.steps
-    layer_pdl_ms = {}
-    for T in Ts:
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        x, lg = dev_in[T][0]
-        layer(x, lg, out=outs[T])
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(args.steps):
-            x, lg = dev_in[T][i % NBATCH]
-            layer(x, lg, out=outs[T])
-        e1.record(stream)
-        torch.cuda.synchronize()
-        layer_pdl_ms[T] = e0.elapsed_time(e1) / args.steps
-    fp8 = dtype == 1
-    gu_bytes = {T: statistics.mean(gate_up_bytes(T, k, H, I, a, fp8) for a in active[T])
-                for T in Ts}
-    hbm, tf, src = peaks()
-    tpeak = tf * (2 if fp8 else 1)   # e4m3 dense peak = 2x the measured bf16 peak (nominal ratio)
-    # dominant kernel: the gate/up GEMM; its largest launch (the largest T)
-    Tr = max(Ts)
-    gu_flops = {T: 4.0 * T * k * H * I for T in Ts}      # 2 GEMMs of 2*H*I per assignment
-    kname = "grouped_gemm_kernel<%s, gate/up> at T=%d" % ("e4m3" if fp8 else "bf16", Tr)
-    if WORKLOADS[args.workload]["bound"] == "hbm":
-        achieved = gu_bytes[Tr] / (gu_ms[Tr] / 1e3) / 1e9
-        agg = sum(gu_bytes[T] for T in Ts) / (sum(gu_ms[T] for T in Ts) / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4),
-                    "traffic": TRAFFIC.get((args.workload, Tr)), "kernel": kname,
-                    "bytes_per_launch": int(gu_bytes[Tr]),
-                    "all_T_achieved": round(agg, 1), "all_T_frac": round(agg / hbm, 4),
-                    "peak_source": src}
-    else:
-        achieved = gu_flops[Tr] / (gu_ms[Tr] / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak,
-                    "unit": "TFLOP/s", "frac": round(achieved / tpeak, 4),
-                    "traffic": TRAFFIC.get((args.workload, Tr)), "kernel": kname,
-                    "flops_per_launch": int(gu_flops[Tr]),
-                    "peak_source": src + (" (bf16 burst x2 for e4m3)" if fp8 else " (bf16 burst)")}
-    wb = 1 if fp8 else 2
-    per_T = {}
-    for T in Ts:
-        a = statistics.mean(active[T])
-        layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
-        layer_flops = 6.0 * T * k * H * I
-        lt = layer_graph_ms.get(T, layer_pdl_ms[T])
-        per_T[str(T)] = {"layer_us": round(1e3 * lt, 2),
-                         "layer_us_direct": round(1e3 * layer_pdl_ms[T], 2),
-                         "cuda_graph": T in graphs,
-                         "layer_tflops": round(layer_flops / (lt / 1e3) / 1e12, 1),
-                         "layer_tensor_frac": round(layer_flops / (lt / 1e3) / 1e12 / tpeak, 4),
-                         "layer_us_staged": round(1e3 * layer_ms[T], 2),
-                         "gate_up_us": round(1e3 * gu_ms[T], 2),
-                         "down_us": round(1e3 * dn_ms[T], 2),
-                         "active_experts": a,
-                         "layer_hbm_gbs": round(layer_bytes / (lt / 1e3) / 1e9, 1),
-                         "layer_hbm_frac": round(layer_bytes / (lt / 1e3) / 1e9 / hbm, 4)}
+            a = statistics.mean(self.active[T])
+            layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
+            layer_flops = 6.0 * T * k * H * I
+            lt = r["layer_graph_ms"].get(T, r["layer_direct_ms"][T])
+            per_T[str(T)] = {
+                "layer_us": round(1e3 * lt, 2),
+                "layer_us_direct": round(1e3 * r["layer_direct_ms"][T], 2),
+                "cuda_graph": T in self.graphs,
+                "tokens_per_s": round(T / (lt / 1e3), 1),
+                "layer_tflops": round(layer_flops / (lt / 1e3) / 1e12, 1),
+                "layer_tensor_frac": round(layer_flops / (lt / 1e3) / 1e12 / tpeak, 4),
+                "layer_hbm_gbs": round(layer_bytes / (lt / 1e3) / 1e9, 1),
+                "layer_hbm_frac": round(layer_bytes / (lt / 1e3) / 1e9 / hbm, 4),
+                "layer_us_staged": round(1e3 * r["layer_ms"][T], 2),
+                "gate_up_us": round(1e3 * gu_ms[T], 2),
+                "gate_up_tensor_frac": round(gu_flops[T] / (gu_ms[T] / 1e3) / 1e12 / tpeak, 4),
+                "gate_up_hbm_frac": round(gu_bytes[T] / (gu_ms[T] / 1e3) / 1e9 / hbm, 4),
+                "down_us": round(1e3 * r["dn_ms"][T], 2),
+                "active_experts": a}
+        return roofline, per_T
 
-    # end to end through the public call, host buffers, copies in the timed
-    # region.  Uploads and read-backs run on two streams of their own,
-    # double-buffered: the inputs of the next layer call go up while the
-    # current one computes, and each output comes back while the next computes.  Every step still moves all
-    # of its inputs and outputs across PCIe inside the timed region.
-    e2e = None
-    if not args.no_e2e:
-        hx = {T: [x.pin_memory() for x, _ in batches[T]] for T in Ts}
-        hl = {T: [lg.pin_memory() for _, lg in batches[T]] for T in Ts}
+    def e2e(self):
+        """End to end through the public call, host buffers, copies in the timed
+        region.  Uploads and read-backs run on two streams of their own,
+        double-buffered: the inputs of the next layer call go up while the
+        current one computes, and each output comes back while the next
+        computes.  Every step still moves all of its inputs and outputs across
+        PCIe inside the timed region."""
+        args, dev, Ts, H, E = self.args, self.dev, self.Ts, self.H, self.E
+        hx = {T: [x.pin_memory() for x, _ in self.batches[T]] for T in Ts}
+        hl = {T: [lg.pin_memory() for _, lg in self.batches[T]] for T in Ts}
         ho = {T: [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
               for T in Ts}
         dx = {T: [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
@@ -471,7 +567,7 @@ def run_native(args):
               for T in Ts}
         h2d = torch.cuda.Stream(device=dev)
         d2h = torch.cuda.Stream(device=dev)
-        jobs = [(T, i) for i in range(args.steps) for T in Ts]
+        stream, layer = self.stream, self.layer
 
         def run_jobs(jobs, start=None):
             """Pipelined H2D -> layer -> D2H over the job list; on return the
@@ -513,44 +609,96 @@ def run_native(args):
                 stream.wait_event(bk)
 
         run_jobs([(T, i) for i in range(args.warmup) for T in Ts])
-        if dist:
-            dist.barrier()
+        if self.dist:
+            self.dist.barrier()
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        run_jobs(jobs, start=a0)
+        run_jobs([(T, i) for i in range(args.steps) for T in Ts], start=a0)
         a1.record(stream)
         torch.cuda.synchronize()
-        _, e_val = aggregate_over_ranks(a0.elapsed_time(a1), tokens_per_step, args.steps, world,
-                                        dist if world > 1 else None, dev)
-        e2e = {"value": e_val,
-               "unit": "tokens/s",
-               "h2d_bytes_per_step": sum(T * H * 2 + T * E * 4 for T in Ts),
-               "d2h_bytes_per_step": sum(T * H * 2 for T in Ts),
-               "copies": "pinned host buffers; uploads and read-backs on two streams, "
-                         "double-buffered"}
+        self.check()
+        _, e_val = aggregate_over_ranks(a0.elapsed_time(a1), sum(Ts), args.steps, self.world,
+                                        self.dist, dev)
+        return {"value": e_val,
+                "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(T * H * 2 + T * E * 4 for T in Ts),
+                "d2h_bytes_per_step": sum(T * H * 2 for T in Ts),
+                "copies": "pinned host buffers; uploads and read-backs on two streams, "
+                          "double-buffered"}
 
+    def launches(self):
+        return self.args.steps * sum(kernels_per_forward(T, self.k, self.fp8, self.H)
+                                     for T in self.Ts)
+
+
+def run_native(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    uuid = torch.cuda.get_device_properties(dev).uuid
+    clk = ClockSampler(uuid).__enter__()
+    atexit.register(clk.__exit__, None, None, None)   # stop the sampler on any exit path
+    head = headline_name(args)
+    Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else None
+
+    b = Bench(head, args, dev, dist, world, Ts)
+    r = b.measure(clk)
+    clk.__exit__(None, None, None)
+    head_clocks = clk.summary()
+    roofline, per_T = b.report(r)
+    e2e = None if args.no_e2e else b.e2e()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, what = oracle_sample(W, dtype, Ts)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what}
+        T, pool = ORACLE_SAMPLE[head]
+        cpu = cpu_baseline(b.W, b.dtype, T, args.cpu_seconds, pool)
+    line = {"metric": "fused-MoE layer tokens/s", "value": r["value"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": r["elapsed_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if b.fp8 else "bf16",
+            "data": "synthetic (seeded; random-init weights of the workload's shape)",
+            "config": {"workload": describe(head), "global_batch": sum(b.Ts) * world,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: expert weights "
+                             f"{3 * b.E * b.H * b.I * (1 if b.fp8 else 2) / 1e9:.2f} GB, "
+                             f"{NBATCH} rotating batches",
+                       "cuda_graphs": sorted(b.graphs) if b.graphs else (b.graph_note or "none"),
+                       "per_T": per_T},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": b.launches(), "clocks": head_clocks}
+    b.release()
 
-    launches = args.steps * sum(kernels_per_forward(T, k, fp8, H) for T in Ts)
+    if args.workload == "all":
+        blocks = {}
+        for name in [n for n in WORKLOADS if n != head]:
+            c = ClockSampler(uuid).__enter__()
+            wb = Bench(name, args, dev, dist, world)
+            rr = wb.measure(c)
+            c.__exit__(None, None, None)
+            rl, pt = wb.report(rr)
+            blk = {"workload": describe(name), "value": rr["value"], "unit": "tokens/s",
+                   "ms_per_step": rr["elapsed_ms"] / args.steps,
+                   "dtype": "fp8" if wb.fp8 else "bf16", "roofline": rl, "per_T": pt,
+                   "cuda_graphs": sorted(wb.graphs) if wb.graphs else (wb.graph_note or "none"),
+                   "gpu_launches": wb.launches(), "clocks": c.summary()}
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                T, pool = ORACLE_SAMPLE[name]
+                blk["cpu_baseline"] = cpu_baseline(wb.W, wb.dtype, T, args.cpu_seconds_other,
+                                                   pool, single_thread=False)
+            wb.release()
+            del wb
+            blocks[name] = blk
+        line["workloads"] = blocks
     if rank == 0:
-        line = {"metric": "fused-MoE layer tokens/s", "value": value, "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if fp8 else "bf16",
-                "data": "synthetic (seeded; random-init weights of the workload's shape)",
-                "config": {"workload": describe(args.workload), "global_batch": sum(Ts) * world,
-                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                           "l2": "inputs larger than L2: expert weights "
-                                 f"{3 * E * H * I * wb / 1e9:.2f} GB, {NBATCH} rotating batches",
-                           "cuda_graphs": sorted(graphs) if graphs else (graph_note or "none"),
-                           "per_T": per_T},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -563,13 +711,20 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS), default="all",
+                    help="all: decode headline plus a block per other workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graphs", action="store_true",
                     help="launch every T directly (no CUDA graphs for T <= 64)")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="oracle budget of the headline's CPU baseline (each of all-core "
+                         "and single-thread)")
+    ap.add_argument("--cpu-seconds-other", type=float, default=3.0,
+                    help="oracle budget of each other workload's CPU baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
-    ap.add_argument("--Ts", default="", help="comma-separated subset of the token counts")
+    ap.add_argument("--Ts", default="", help="comma-separated subset of the headline's "
+                                            "token counts")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -28,7 +28,12 @@
  *   - T = 0 is a valid no-op.
  *   - Limits: 1 <= k <= E <= 256; H and I multiples of 64; block_m a multiple
  *     of 16 (the token granularity of the tensor-core tiles).
- *   - No global state: calls on different streams may run concurrently.
+ *   - Process-wide state is limited to two things: the per-device opt-in of
+ *     the GEMM kernels to more than 48 KB of shared memory (set on the first
+ *     launch on each device, read-only afterwards), and the fixed scratch
+ *     array of moe_align_permute_noalloc (see its entry).  Apart from
+ *     moe_align_permute_noalloc, calls on different streams with separate
+ *     buffers may run concurrently.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

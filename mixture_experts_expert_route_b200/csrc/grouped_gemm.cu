@@ -766,16 +766,36 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, long tiles, int kps) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The opt-in to more than 48 KB of dynamic shared memory is a function
+// attribute held by each device's context, so it is set once per device and
+// per kernel instantiation: a process that drives several GPUs must opt in on
+// each of them.
+constexpr int kMaxDevices = 64;
+
+template <bool FP8, int EPI, bool PAIR>
+cudaError_t opt_in_smem() {
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t err[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    // Every launch asks for at most kDynSmemMax bytes (see the stage count
+    // below); the 1 KB margin in it covers the compiler's padding of the
+    // static shared block.
+    std::call_once(once[dev], [dev] {
+        err[dev] = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, EPI, PAIR>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmemMax);
+    });
+    return err[dev];
+}
+
 template <bool FP8, int EPI, bool PAIR>
 cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b128, const CUtensorMap& b64,
                      const CUtensorMap& b16, const GemmArgs& g, int grid, int smem,
                      cudaStream_t s) {
     auto kern = grouped_gemm_kernel<FP8, EPI, PAIR>;
-    // Every launch asks for at most kDynSmemMax bytes (see the stage count
-    // below); the 1 KB margin in it covers the compiler's padding of the
-    // static shared block.
-    static cudaError_t attr = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmemMax);
+    const cudaError_t attr = opt_in_smem<FP8, EPI, PAIR>();
     if (attr != cudaSuccess) return attr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

@@ -11,9 +11,11 @@
 // Properties a caller must know:
 //   * the array holds kScratchInts int32 counters (256 KB) on every GPU that
 //     loads the library, until the process exits;
-//   * it bounds the problem: ceil(T*k / 2048) * E <= kScratchInts, i.e.
-//     T*k <= 2048 * floor(65536 / E); larger problems return MOE_ERR_WORKSPACE
-//     and launch nothing;
+//   * it bounds the problem: up to T*k = 2048 one CTA does the whole
+//     permutation and needs no scratch; above that the assignments are cut
+//     into chunks of 512 and ceil(T*k / 512) * E <= kScratchInts must hold,
+//     i.e. T*k <= 512 * floor(65536 / E); larger problems return
+//     MOE_ERR_WORKSPACE and launch nothing;
 //   * the first call on a device looks up the array's device address
 //     (cudaGetSymbolAddress) once for that device; make that first call before
 //     any stream capture;

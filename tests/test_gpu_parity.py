@@ -190,9 +190,71 @@ def test_forward_block_m_variants(moe, block_m):
 
 def test_forward_deterministic(moe):
     L = make_layer("tiny", T=200, E=8, k=2, H=256, I=256, seed=2)
-    outs = [run_forward(moe, 0, L, max_ctas=11)[0] for _ in range(3)]
+    outs = [run_forward(moe, 0, L, max_ctas=11)[0] for _ in range(10)]
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
+
+
+def test_fp8_zero_input(moe):
+    """x = 0: amax = 0 gives s_x = 1 (and then h = 0, s_h = 1); the output is
+    exactly zero, as the oracle's."""
+    L = make_layer("tiny", T=24, E=8, k=2, H=256, I=256, seed=3)
+    L.x = torch.zeros_like(L.x)
+    out, ids, w = run_forward(moe, 1, L)
+    ids_o, w_o = check_routing(ids, w, L.logits)
+    g, u, d = L.weights_bf16()
+    ref, _, (sx, sh) = oracle.moe_layer_fp8(L.x, ids_o, w_o, g, u, d)
+    assert sx == 1.0 and sh == 1.0 and not ref.any()
+    assert torch.count_nonzero(out).item() == 0
+
+
+# bf16 values a for which the fp32 product a * (1 / (a / 448)) rounds above
+# 448: the element equal to amax(x) must still get the largest code (448).
+@pytest.mark.parametrize("amax", [8.1875, 11.25, 15.9375])
+def test_fp8_amax_element_saturates(moe, amax):
+    L = make_layer("tiny", T=48, E=8, k=2, H=256, I=256, seed=4)
+    x = L.x.clone()
+    x[3, 17] = amax
+    x[20, 200] = -amax
+    x[41, 5] = amax
+    L.x = x
+    out, ids, w = run_forward(moe, 1, L)
+    ids_o, w_o = check_routing(ids, w, L.logits)
+    g, u, d = L.weights_bf16()
+    ref, _, (sx, _) = oracle.moe_layer_fp8(L.x, ids_o, w_o, g, u, d)
+    assert sx == np.float32(np.float32(amax) / np.float32(448.0))
+    assert torch.isfinite(out).all()
+    assert_close(out, ref, 1, f"planted amax {amax}")
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_nonfinite_logits(moe, dtype):
+    """Tokens with NaN, -inf and +inf logits: routing stays bit-exact (NaN
+    ranks last, -inf below every number); a +inf selection makes that token's
+    weights NaN (exp(inf - inf)) on both sides, and only that token's output;
+    every other token matches the oracle."""
+    L = make_layer("tiny", T=40, E=8, k=2, H=256, I=256, seed=8)
+    lg = L.logits.clone()
+    lg[5, 3] = float("nan")
+    lg[6, 0] = float("nan")
+    lg[6, 7] = float("nan")
+    lg[7, 2] = float("-inf")
+    lg[8, :6] = float("-inf")            # two finite logits left: they are chosen
+    lg[9, 4] = float("inf")
+    L.logits = lg
+    out, ids, w = run_forward(moe, dtype, L)
+    ids_o, w_o = check_routing(ids, w, lg)
+    bad = ~np.isfinite(w_o).all(axis=1)
+    assert bad.tolist() == [t == 9 for t in range(L.T)]
+    assert torch.isnan(w[9]).all()
+    good = [t for t in range(L.T) if not bad[t]]
+    g, u, d = L.weights_bf16()
+    # the oracle on the other tokens (token 9's NaN weights zeroed: they do not
+    # enter any other token's output, nor the FP8 scale of h)
+    w_fin = np.where(np.isfinite(w_o), w_o, 0.0)
+    ref = oracle_layer(dtype, L.x, ids_o, w_fin, g, u, d, tokens=good)
+    assert_close(out[good], ref, dtype, f"non-finite logits dtype={dtype}")
+    assert not torch.isfinite(out[9]).any()
 
 
 def test_forward_empty_batch(moe):
