@@ -4,8 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all]
                     [--impl native|reference]
 
-A step is one pass of the whole layer (route -> permute -> gather -> gate/up
-GEMM -> [FP8 h quant] -> down GEMM -> combine) over one
+A step is one pass of the whole layer (route -> permute -> gate/up GEMM with
+the gather of x fused in -> [FP8 h quant] -> down GEMM -> combine) over one
 batch of every token count of a workload, e.g. T = 1, 4, 16, 64 for the
 decode workload (H=4096, I=14336, E=8, top-2, bf16).  Inputs are seeded
 synthetic tensors; the expert weights are larger than the 126 MB L2 and four
@@ -89,18 +89,18 @@ def describe(name):
 
 
 def kernels_per_forward(T, k, fp8, H):
-    """Kernels one moe_forward launches (the cudaMemsetAsync is not a kernel)."""
+    """Kernels one moe_forward launches."""
     A = T * k
     small = T <= SMALL_T and A <= CHUNK
     if small:
         n = 1                                   # fused route + permute
     else:
         n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
-    n += 1                                      # gather
-    n += 1 if fp8 and not (small and T * H <= SMALL_AMAX) else 0   # amax(x)
-    n += 1                                      # gate/up GEMM
+    # FP8: amax(x) and the codes of x (in the route kernel for small batches)
+    n += 2 if fp8 and not (small and T * H <= SMALL_AMAX) else 0
+    n += 1                                      # gate/up GEMM (gathers x itself)
     n += 1 if fp8 else 0                        # h quantisation
-    n += 2                                      # down GEMM + combine
+    n += 2                                      # down GEMM + combine (or finalize)
     return n
 
 

@@ -165,11 +165,14 @@ MOE_API moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const 
  * SageMaker AI"), computed with the expert-weight rows in the tensor core's
  * M slot and the tokens in N (the operand swap of "A mátrixok felcserélése
  * jobban kihasználja a Hopper GPU-kat", re-derived for tcgen05), with the
- * SiLU*up and routing-weight epilogues fused in:
- *   X_perm[p] = x[sorted_ids[p] / k]      (zero for pads; FP8: quantised
- *                                           with s_x = amax(x)/448)
- *   h[p]      = SiLU(X_perm[p] W_g[e]) * (X_perm[p] W_u[e])   (bf16; FP8:
- *                                           then quantised with s_h)
+ * gather of the token rows, the SiLU*up and the routing-weight epilogues
+ * fused in:
+ *   X_p       = x[sorted_ids[p] / k]      gathered by the gate/up GEMM's
+ *                                         operand loads, never stored (zero for
+ *                                         pads; FP8: the e4m3 codes of x with
+ *                                         s_x = amax(x)/448, made in token order)
+ *   h[p]      = SiLU(X_p W_g[e]) * (X_p W_u[e])   (bf16; FP8: then quantised
+ *                                                  with s_h)
  *   y_perm[p] = w[sorted_ids[p]] * (h[p] W_d[e])   (bf16; 0 for pads)
  * for every row p of expert e's block.  Inputs come from moe_align_permute.
  * FP8 activations are coded as RNE_sat(v * (1/s)) with the fp32 reciprocal of
@@ -222,11 +225,27 @@ MOE_API moe_status moe_combine(const void* y_perm, const int32_t* inv_perm, int 
  *   status   optional device status word (NULL: the first int32 of ws)
  *   block_m  0 selects 16
  *   events / n_events  optional: if non-NULL, events[i] is recorded on the
- *            stream after stage i (0 entry, 1 route+permute, 2 gather/quant,
- *            3 gate/up GEMM, 4 h quant (FP8), 5 down GEMM, 6 combine); used to
- *            time the stages.  n_events must be 7 when events is non-NULL.
+ *            stream after stage i (0 entry, 1 route+permute, 2 FP8 x
+ *            quantisation (empty for bf16 and small FP8 batches, where the
+ *            route kernel does it), 3 gate/up GEMM, 4 h quant (FP8), 5 down
+ *            GEMM, 6 combine or finalize); used to time the stages.  n_events
+ *            must be 7 when events is non-NULL.
+ *   combine  a moe_combine_mode (0 = auto).
  * Errors: as for the stages above.
  */
+/* How moe_forward forms out[t] = sum_j y(t, j) (a7). */
+typedef enum {
+    MOE_COMBINE_AUTO = 0,          /* fused for T*k >= 4096, deterministic below */
+    MOE_COMBINE_DETERMINISTIC = 1, /* the down GEMM writes y_perm rows (bf16); a
+                                      combine kernel sums each token's k rows in
+                                      fp32 in j order: bit-reproducible */
+    MOE_COMBINE_FUSED = 2          /* the down GEMM's epilogue adds w*y (fp32)
+                                      into a token-order accumulator, converted
+                                      to bf16 at the end: no y_perm round trip,
+                                      but the summation order follows the
+                                      schedule, so the last bit may vary */
+} moe_combine_mode;
+
 typedef struct {
     moe_dtype dtype;
     int T, k, E, H, I;
@@ -242,6 +261,7 @@ typedef struct {
     int max_ctas;
     moe_event_t* events;
     int n_events;
+    int combine;               /* a moe_combine_mode */
 } moe_forward_args;
 
 MOE_API size_t moe_forward_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,

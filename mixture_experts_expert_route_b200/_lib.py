@@ -13,9 +13,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+# MOE_B200_DEBUG_CHECKS=1 selects the build whose kernels validate the
+# permutation they are handed (see build.py --debug-checks)
+DEBUG_CHECKS = os.environ.get("MOE_B200_DEBUG_CHECKS", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libmoe_b200_debug.so" if DEBUG_CHECKS else "libmoe_b200.so")
 
 BF16, FP8_E4M3 = 0, 1
+COMBINE_AUTO, COMBINE_DETERMINISTIC, COMBINE_FUSED = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT",
           6: "MOE_ERR_DEVICE"}
@@ -42,7 +46,7 @@ class ForwardArgs(ctypes.Structure):
     _fields_ = [("dtype", I32), ("T", I32), ("k", I32), ("E", I32), ("H", I32), ("I", I32),
                 ("block_m", I32), ("x", P), ("logits", P), ("packed", P), ("scales", P),
                 ("out", P), ("ids", P), ("w", P), ("status", P), ("max_ctas", I32),
-                ("events", P), ("n_events", I32)]
+                ("events", P), ("n_events", I32), ("combine", I32)]
 
 
 _SIGS = {
@@ -217,9 +221,10 @@ def forward_workspace_size(dtype, T, k, E, H, I, block_m=0) -> int:
 
 def forward(dtype: int, x, logits, packed, scales, E: int, I: int, k: int, out=None, ids=None,
             w=None, status=None, ws=None, block_m: int = 0, max_ctas: int = 0, events=None,
-            stream=None):
+            combine: int = COMBINE_AUTO, stream=None):
     """The whole layer.  ``events`` (7 torch.cuda.Event, optional) are recorded after
-    each stage: entry, route+permute, gather, gate/up, h quant, down, combine."""
+    each stage: entry, route+permute, FP8 x quantisation, gate/up, h quant, down,
+    combine.  ``combine``: COMBINE_AUTO, COMBINE_DETERMINISTIC or COMBINE_FUSED."""
     T, H = x.shape
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     n = forward_workspace_size(dtype, T, k, E, H, I, block_m)
@@ -236,7 +241,7 @@ def forward(dtype: int, x, logits, packed, scales, E: int, I: int, k: int, out=N
     a = ForwardArgs(dtype, T, k, E, H, I, block_m, _ptr(x), _ptr(logits), _ptr(packed),
                     _ptr(scales), _ptr(out), _ptr(ids), _ptr(w), _ptr(status), max_ctas,
                     ctypes.cast(ev_arr, ctypes.c_void_p) if ev_arr is not None else None,
-                    7 if ev_arr is not None else 0)
+                    7 if ev_arr is not None else 0, combine)
     _check(lib().moe_forward(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return out
@@ -259,9 +264,10 @@ class MoELayer:
     """
 
     def __init__(self, Wg, Wu, Wd, k: int, dtype: int = BF16, block_m: int = 0,
-                 max_ctas: int = 0):
+                 max_ctas: int = 0, combine: int = COMBINE_AUTO):
         self.E, self.H, self.I = Wg.shape
         self.k, self.dtype, self.block_m, self.max_ctas = k, dtype, block_m, max_ctas
+        self.combine = combine
         self.packed, self.scales = pack_weights(dtype, Wg, Wu, Wd)
         self.device = Wg.device
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
@@ -279,7 +285,7 @@ class MoELayer:
         return forward(self.dtype, x, logits, self.packed, self.scales, self.E, self.I,
                        self.k, out=out, status=self.status, ws=self.workspace(T),
                        block_m=self.block_m, max_ctas=self.max_ctas, events=events,
-                       stream=stream)
+                       combine=self.combine, stream=stream)
 
     def check(self) -> int:
         return check_status(self.status)

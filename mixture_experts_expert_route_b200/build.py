@@ -1,6 +1,11 @@
 """Builds libmoe_b200.so in-tree with nvcc for sm_100a.
 
-    python -m mixture_experts_expert_route_b200.build [--verbose-ptxas]
+    python -m mixture_experts_expert_route_b200.build [--verbose-ptxas] [--debug-checks]
+
+--debug-checks builds libmoe_b200_debug.so instead: the same library compiled
+with MOE_DEBUG_CHECKS, whose kernels validate the permutation they are handed
+and report a bad entry in the status word (MOE_ERR_DEVICE).  The binding
+loads it when the environment sets MOE_B200_DEBUG_CHECKS=1.
 """
 from __future__ import annotations
 
@@ -15,6 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["route_permute.cu", "elementwise.cu", "grouped_gemm.cu", "moe_api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 LIB = os.path.join(HERE, "libmoe_b200.so")
+LIB_DEBUG = os.path.join(HERE, "libmoe_b200_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -25,22 +31,29 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def lib_path(debug: bool = False) -> str:
+    return LIB_DEBUG if debug else LIB
+
+
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "moe.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(ROOT, "_build")
+def build(force: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    lib = lib_path(debug)
+    if not force and not _stale(lib):
+        return lib
+    objdir = os.path.join(ROOT, "_build", "debug" if debug else "release")
     os.makedirs(objdir, exist_ok=True)
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                     "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
+    if debug:
+        flags += ["-DMOE_DEBUG_CHECKS"]
     if ptxas_verbose:
         flags += ["-Xptxas", "-v"]
     objs = []
@@ -48,12 +61,12 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         subprocess.check_call([nvcc(), *flags, "-c", os.path.join(CSRC, src), "-o", obj])
         objs.append(obj)
-    tmp = LIB + f".{os.getpid()}.tmp"
+    tmp = lib + f".{os.getpid()}.tmp"
     subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                debug="--debug-checks" in sys.argv))

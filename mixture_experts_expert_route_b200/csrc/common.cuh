@@ -13,6 +13,16 @@
 
 namespace moe {
 
+// Debug builds (-DMOE_DEBUG_CHECKS) validate the permutation a kernel is
+// handed (offsets within the capacity, flat indices within T*k) on the
+// device: a bad entry is recorded as MOE_ERR_DEVICE in the status word and
+// treated as a pad, never trapped.  Release builds trust their inputs.
+#ifdef MOE_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
 constexpr int kMaxExperts = 256;
 constexpr int kMaxCtas = 256;          // upper bound on the persistent grid
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: no healthy wait comes close
@@ -76,6 +86,74 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (abort && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// Arrive with release semantics at cluster scope, on a barrier in this CTA or
+// (shared::cluster address) in the other CTA of the pair: orders this
+// thread's prior memory operations (and what it acquired) before the arrival
+// for a waiter in either CTA.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// try_wait with acquire semantics at cluster scope (the arrivals may come from
+// the other CTA of a pair).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// ------------------------------------------------------------------ cp.async
+// 16-byte global -> shared copy through L2 (no L1 allocation).  src_bytes = 0
+// reads nothing and writes 16 zero bytes.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gmem_src,
+                                           uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gmem_src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// One arrive-on for *bar once every cp.async this thread issued so far has
+// completed (the barrier's expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Makes shared-memory writes of the generic proxy (st.shared, cp.async) that
+// this thread performed or acquired visible to the async proxy (tensor-core
+// operand reads, bulk copies) that follows.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Fire-and-forget fp32 add in global memory (performed at L2).
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
 // ------------------------------------------------------------------ PDL
@@ -308,6 +386,46 @@ __device__ __forceinline__ float fp8_scale_from_amax(uint32_t bits) {
 // Round-to-nearest-even, saturating e4m3 code of x / s.
 __device__ __forceinline__ uint8_t fp8_quant(float x, float s) {
     return static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x, s), __NV_SATFINITE, __NV_E4M3));
+}
+
+// ------------------------------------------------------------------ bf16 / e4m3 vectors
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ float amax8(uint4 v) {
+    float m = 0.0f;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    return m;
+}
+
+// Activations: e4m3 codes of 8 packed bf16 values times inv_s = 1/s (the
+// weights, quantised once, keep the correctly rounded x / s).  Scaling by the
+// reciprocal costs one multiply where an IEEE division took most of the
+// kernel's issue slots; a code can differ by one step from RNE(x / s) only
+// when x / s lies within an fp32 ulp of an e4m3 rounding midpoint.  Two
+// values per saturating RNE conversion.  A scale so small that 1/s overflows
+// (amax below ~1e-36) takes the division instead (0 * inf would be NaN).
+__device__ __forceinline__ uint2 quant8(uint4 v, float inv_s, float s) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0, 0};
+    if (!(inv_s <= 3.0e38f)) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = fp8_quant(bf16_lo(w[i]), s);
+            const uint32_t hi = fp8_quant(bf16_hi(w[i]), s);
+            out[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+        }
+        return make_uint2(out[0], out[1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = make_float2(bf16_lo(w[i]) * inv_s, bf16_hi(w[i]) * inv_s);
+        const uint32_t pair = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        out[i >> 1] |= pair << (16 * (i & 1));
+    }
+    return make_uint2(out[0], out[1]);
 }
 
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }

@@ -1,8 +1,9 @@
-// elementwise.cu -- the layer's memory-bound steps: a3 gather (+ FP8
-// quantisation of x), a5 FP8 quantisation of h, a7 combine, the one-time
-// weight packing, and the failure-detection self-test.  All are HBM-bound:
-// 16-byte vector accesses, one vector per thread (one warp per row for large
-// bf16 gathers), grids sized from the data.
+// elementwise.cu -- the layer's memory-bound steps around the GEMMs: the FP8
+// quantisation of x (a3; its gather is fused into the gate/up GEMM's operand
+// loads) and of h (a5), the combine (a7: the deterministic gather-sum, or the
+// conversion of the fused fp32 accumulator), the one-time weight packing, and
+// the failure-detection self-test.  All are HBM-bound: 16-byte vector
+// accesses, one vector per thread, grids sized from the data.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -12,91 +13,10 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Flat element-parallel mapping for the row-wise kernels below: vector i of
-// the used rows (row i / vpr, 16-byte vector i % vpr) per thread.  One warp
-// per row would leave a small batch (a few dozen rows) with a few dozen
-// warps, each walking its row one dependent load at a time; measured on
-// B200, FP8 T = 1: gather 12.3 -> 4.8 us, h quantisation 25.2 -> 4.9 us.
-// Large bf16 batches (capacity >= kRowGatherMinRows) keep one warp per row,
-// which measured faster there (prefill T = 4096: 12 us less per layer).
+// One 16-byte vector per thread: a small batch still has thousands of loads
+// in flight (measured on B200, FP8 T = 1: h quantisation 25.2 -> 4.9 us
+// against one warp per row).
 constexpr int kVecBlocksPerSm = 8;
-constexpr int kRowGatherMinRows = 16384;
-constexpr int kRowsPerBlock = kThreads / 32;
-
-__global__ void __launch_bounds__(kThreads)
-    gather_bf16_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
-                            const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
-                            int capacity, const float* __restrict__ w, uint4* __restrict__ x_perm,
-                            float* __restrict__ w_perm) {
-    pdl_wait();
-    pdl_trigger();
-    const int p = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (p >= capacity || p >= offsets[E]) return;
-    const int sid = sorted_ids[p];
-    if (lane == 0) w_perm[p] = sid >= 0 ? w[sid] : 0.0f;
-    uint4* dst = x_perm + static_cast<long>(p) * vec_per_row;
-    if (sid < 0) {
-        for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
-        return;
-    }
-    const uint4* src = x + static_cast<long>(sid / k) * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
-}
-
-// Row/vector position of flat index i (row p, 16-byte vector v of a row of
-// vpr vectors), advanced through a grid-stride loop by additions only: the
-// per-element 64-bit division it replaces dominated the kernels' issue slots.
-struct RowVec {
-    int p, v, sq, sr, vpr;
-    __device__ __forceinline__ RowVec(long i0, long stride, int vpr_) : vpr(vpr_) {
-        p = static_cast<int>(i0 / vpr);
-        v = static_cast<int>(i0 - static_cast<long>(p) * vpr);
-        sq = static_cast<int>(stride / vpr);
-        sr = static_cast<int>(stride - static_cast<long>(sq) * vpr);
-    }
-    __device__ __forceinline__ void next() {
-        p += sq;
-        v += sr;
-        if (v >= vpr) {
-            v -= vpr;
-            ++p;
-        }
-    }
-    __device__ __forceinline__ long flat() const { return static_cast<long>(p) * vpr + v; }
-};
-
-// a3: X_perm[p] = x[sorted_ids[p] / k] for p < offsets[E]; pad rows are zero.
-// Also w_perm[p] = w[sorted_ids[p]] (0 for pads), the routing weight the down
-// GEMM's epilogue applies to row p.
-__global__ void __launch_bounds__(kThreads)
-    gather_bf16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
-                       const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
-                       int capacity, const float* __restrict__ w, uint4* __restrict__ x_perm,
-                       float* __restrict__ w_perm) {
-    pdl_wait();
-    pdl_trigger();
-    const int rows = min(capacity, offsets[E]);
-    for (RowVec r(static_cast<long>(blockIdx.x) * kThreads + threadIdx.x,
-                  static_cast<long>(gridDim.x) * kThreads, vec_per_row);
-         r.p < rows; r.next()) {
-        const int sid = sorted_ids[r.p];
-        if (r.v == 0) w_perm[r.p] = sid >= 0 ? w[sid] : 0.0f;
-        x_perm[r.flat()] = sid >= 0 ? x[static_cast<long>(sid / k) * vec_per_row + r.v]
-                                    : make_uint4(0, 0, 0, 0);
-    }
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-
-__device__ __forceinline__ float amax8(uint4 v) {
-    float m = 0.0f;
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    return m;
-}
 
 // amax over n bf16 values (n % 8 == 0), folded into *amax_bits with atomicMax.
 __global__ void __launch_bounds__(kThreads)
@@ -118,54 +38,18 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// Activations: e4m3 codes of 8 packed bf16 values times inv_s = 1/s (the
-// weights, quantised once, keep the correctly rounded x / s).  Scaling by the
-// reciprocal costs one multiply where an IEEE division took most of the
-// kernel's issue slots; a code can differ by one step from RNE(x / s) only
-// when x / s lies within an fp32 ulp of an e4m3 rounding midpoint.  Two
-// values per saturating RNE conversion.  A scale so small that 1/s overflows
-// (amax below ~1e-36) takes the division instead (0 * inf would be NaN).
-__device__ __forceinline__ uint2 quant8(uint4 v, float inv_s, float s) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[2] = {0, 0};
-    if (!(inv_s <= 3.0e38f)) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = fp8_quant(bf16_lo(w[i]), s);
-            const uint32_t hi = fp8_quant(bf16_hi(w[i]), s);
-            out[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
-        }
-        return make_uint2(out[0], out[1]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = make_float2(bf16_lo(w[i]) * inv_s, bf16_hi(w[i]) * inv_s);
-        const uint32_t pair = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
-        out[i >> 1] |= pair << (16 * (i & 1));
-    }
-    return make_uint2(out[0], out[1]);
-}
-
-// a3 (FP8): X_perm[p] = e4m3(x[sorted_ids[p] / k] / s_x), s_x = amax(x)/448.
+// a3 (FP8): x in token order -> e4m3 codes with s_x = amax(x)/448; the
+// gate/up GEMM gathers the rows of these codes.
 __global__ void __launch_bounds__(kThreads)
-    gather_fp8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_ids,
-                      const int32_t* __restrict__ offsets, int E, int k, int vec_per_row,
-                      int capacity, const uint32_t* __restrict__ amax_bits,
-                      const float* __restrict__ w, uint2* __restrict__ x_perm,
-                      float* __restrict__ w_perm) {
+    quant_x_fp8_kernel(const uint4* __restrict__ x, long nvec,
+                       const uint32_t* __restrict__ amax_bits, uint2* __restrict__ xq) {
     pdl_wait();
     pdl_trigger();
-    const int rows = min(capacity, offsets[E]);
     const float s = fp8_scale_from_amax(*amax_bits);
     const float inv_s = 1.0f / s;
-    for (RowVec r(static_cast<long>(blockIdx.x) * kThreads + threadIdx.x,
-                  static_cast<long>(gridDim.x) * kThreads, vec_per_row);
-         r.p < rows; r.next()) {
-        const int sid = sorted_ids[r.p];
-        if (r.v == 0) w_perm[r.p] = sid >= 0 ? w[sid] : 0.0f;
-        x_perm[r.flat()] = sid >= 0 ? quant8(x[static_cast<long>(sid / k) * vec_per_row + r.v], inv_s, s)
-                                    : make_uint2(0, 0);
-    }
+    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < nvec;
+         i += static_cast<long>(gridDim.x) * kThreads)
+        xq[i] = quant8(x[i], inv_s, s);
 }
 
 // a5: rows p < offsets[E] of a bf16 matrix -> e4m3 with s = amax/448.
@@ -185,9 +69,10 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // a7: out[t] = sum_j y_perm[inv_perm[t*k + j]] in fp32, j ascending.
+// Debug builds check each slot against the rows of y_perm (when known).
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm, int T,
-                   int k, int vec_per_row, uint4* __restrict__ out) {
+                   int k, int vec_per_row, int rows, int32_t* status, uint4* __restrict__ out) {
     pdl_wait();
     pdl_trigger();
     const long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x;
@@ -200,6 +85,12 @@ __global__ void __launch_bounds__(kThreads)
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
         const int p = inv_perm[t * k + j];
+        if constexpr (kDebugChecks) {
+            if (p < 0 || p >= rows) {
+                report(status, MOE_ERR_DEVICE);
+                continue;
+            }
+        }
         const uint4 q = y[static_cast<long>(p) * vec_per_row + v];
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -215,6 +106,26 @@ __global__ void __launch_bounds__(kThreads)
         o[c] = *reinterpret_cast<const uint32_t*>(&b);
     }
     out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// a7 (fused form): out = bf16(acc), the fp32 token-order sums the down
+// GEMM's epilogue accumulated.
+__global__ void __launch_bounds__(kThreads)
+    finalize_kernel(const float4* __restrict__ acc, long nvec8, uint4* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    for (long i = static_cast<long>(blockIdx.x) * kThreads + threadIdx.x; i < nvec8;
+         i += static_cast<long>(gridDim.x) * kThreads) {
+        const float4 a = acc[2 * i], b = acc[2 * i + 1];
+        const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+        const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
+        const __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+        out[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&p0),
+                            *reinterpret_cast<const uint32_t*>(&p1),
+                            *reinterpret_cast<const uint32_t*>(&p2),
+                            *reinterpret_cast<const uint32_t*>(&p3));
+    }
 }
 
 // ---- weight packing (one-time)
@@ -322,33 +233,17 @@ int vec_blocks(long nvec) { return blocks_for(nvec, kThreads, kVecBlocksPerSm * 
 
 }  // namespace
 
-cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                               int E, int k, int H, int capacity, const float* w, void* x_perm,
-                               float* w_perm, cudaStream_t s) {
-    if (capacity == 0) return cudaSuccess;
-    if (capacity >= kRowGatherMinRows)
-        return launch_pdl(gather_bf16_rows_kernel,
-                          dim3((capacity + kRowsPerBlock - 1) / kRowsPerBlock), dim3(kThreads), 0, s,
-                          static_cast<const uint4*>(x), sorted_ids, offsets, E, k, H / 8, capacity,
-                          w, static_cast<uint4*>(x_perm), w_perm);
-    return launch_pdl(gather_bf16_kernel, dim3(vec_blocks(static_cast<long>(capacity) * (H / 8))),
-                      dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
-                      k, H / 8, capacity, w, static_cast<uint4*>(x_perm), w_perm);
-}
-
 cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s) {
     if (n == 0) return cudaSuccess;
     return launch_pdl(amax_bf16_kernel, dim3(blocks_for(n / 8, kThreads * 4, 1184)),
                       dim3(kThreads), 0, s, static_cast<const uint4*>(src), n / 8, amax_bits);
 }
 
-cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                              int E, int k, int H, int capacity, const uint32_t* amax_bits,
-                              const float* w, void* x_perm, float* w_perm, cudaStream_t s) {
-    if (capacity == 0) return cudaSuccess;
-    return launch_pdl(gather_fp8_kernel, dim3(vec_blocks(static_cast<long>(capacity) * (H / 8))),
-                      dim3(kThreads), 0, s, static_cast<const uint4*>(x), sorted_ids, offsets, E,
-                      k, H / 8, capacity, amax_bits, w, static_cast<uint2*>(x_perm), w_perm);
+cudaError_t launch_quant_x_fp8(const void* x, long n, const uint32_t* amax_bits, void* xq,
+                               cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    return launch_pdl(quant_x_fp8_kernel, dim3(vec_blocks(n / 8)), dim3(kThreads), 0, s,
+                      static_cast<const uint4*>(x), n / 8, amax_bits, static_cast<uint2*>(xq));
 }
 
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
@@ -361,12 +256,18 @@ cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, 
 }
 
 cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
-                           void* out, cudaStream_t s) {
+                           void* out, cudaStream_t s, int rows, int32_t* status) {
     const long n = static_cast<long>(T) * (H / 8);
     if (n == 0) return cudaSuccess;
     return launch_pdl(combine_kernel, dim3(static_cast<unsigned>((n + kThreads - 1) / kThreads)),
                       dim3(kThreads), 0, s, static_cast<const uint4*>(y_perm), inv_perm, T, k,
-                      H / 8, static_cast<uint4*>(out));
+                      H / 8, rows, status, static_cast<uint4*>(out));
+}
+
+cudaError_t launch_finalize(const float* acc, long n, void* out, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    return launch_pdl(finalize_kernel, dim3(vec_blocks(n / 8)), dim3(kThreads), 0, s,
+                      reinterpret_cast<const float4*>(acc), n / 8, static_cast<uint4*>(out));
 }
 
 cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, const void* Wu,

@@ -1,5 +1,7 @@
-// grouped_gemm.cu -- a4 (gate/up GEMM + SiLU*up) and a6 (down GEMM + routing
-// weight) as one persistent, warp-specialised tcgen05 kernel.
+// grouped_gemm.cu -- a4 (gate/up GEMM + SiLU*up, with the gather of x fused
+// into its operand loads) and a6 (down GEMM + routing weight, optionally with
+// the top-k combine fused into its epilogue) as one persistent,
+// warp-specialised tcgen05 kernel.
 //
 // The expert GEMM is A[M,K] x B[K,N] with M = tokens, K = hidden and N = the
 // expert's output size ("Ingénierie de kernels Mixture-of-Experts sur Amazon
@@ -21,9 +23,17 @@
 // whichever contributor arrives last, which sums the fp32 partials in CTA
 // order -- a fixed order, so the result does not depend on timing.
 //
-// Roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (single
-// thread), warp 2 = TMEM allocator, warps 4-11 = epilogue (two warps per
-// 32-lane TMEM quarter, alternating 16-column chunks).
+// Fusion ("one pass, no intermediate global round trips", same section): the
+// gate/up kernel reads its token rows straight from x (token order) by the
+// permutation, so no permuted copy of the activations is written; the down
+// kernel can add w * y into an fp32 accumulator in token order (the combine)
+// instead of writing permuted rows.
+//
+// Roles (512 threads): warp 0 = copy producer (weights; the down kernel's
+// activation rows by TMA), warp 1 = MMA issuer (single thread), warp 2 =
+// TMEM allocator, then (gate/up) the gather forwarder, warps 4-11 = epilogue
+// (two warps per 32-lane TMEM quarter, alternating 16-column chunks), warps
+// 12-15 = gather of the gate/up kernel's token rows (cp.async).
 // Shared-memory ring of stages of KPS k-blocks (A KPS*16 KB + B KPS*rows*128 B,
 // 128-byte swizzle): 2 stages of 4 k-blocks on one CTA (token tiles of at most
 // 64 rows), 3 stages of 2 k-blocks per CTA of a pair (larger tiles).  Two TMEM
@@ -37,11 +47,14 @@
 //
 // Weights (A) are pre-packed as 16 KB tiles that are already the swizzled
 // shared-memory image of one stage, so a stage's A operand (one to four
-// consecutive k-blocks) is one contiguous copy.  Activations (B) come through
-// TMA tensor maps with 128-, 64- and 16-row boxes, so a token tile moves only
-// its own rows.  Launched with programmatic dependent launch: the producer
-// fetches the first weight tiles before waiting for the previous kernel, whose
-// output (B) it loads after.
+// consecutive k-blocks) is one contiguous copy.  The gate/up kernel's token
+// rows (B) are gathered with 16-byte cp.async copies placed in the same
+// swizzled layout (zero-filled for pads); a forwarder thread waits for them,
+// makes them visible to the tensor core's (async) proxy and arrives on the
+// MMA's barrier.  The down kernel's rows (h, already in permuted order) come
+// through TMA tensor maps with 128-, 64- and 16-row boxes.  Launched with
+// programmatic dependent launch: the producer fetches the first weight tiles
+// before waiting for the previous kernel, whose outputs it loads after.
 #include <cstring>
 #include <mutex>
 
@@ -55,10 +68,14 @@ namespace {
 constexpr int kBM = 128;            // weight rows per tile (UMMA M)
 constexpr int kRowBytes = 128;      // K bytes per stage row (one swizzle atom)
 constexpr int kATileBytes = kBM * kRowBytes;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kFwdWarp = 2;           // TMEM allocator, then the gather forwarder
 constexpr int kEpiWarp0 = 4;          // warps 4..11: two per TMEM lane quarter
 constexpr int kEpiThreads = 256;
-constexpr int kMaxStages = 12;
+constexpr int kGatherWarp0 = 12;      // warps 12..15 gather the gate/up token rows
+constexpr int kGatherLanes = 128;
+constexpr int kGatherRowsPerPass = kGatherLanes / 8;   // 8 lanes per 128-byte row
+constexpr int kMaxStages = 4;
 constexpr int kMinKbPerCta = 4;
 constexpr int kStagingBytes = 8 * 1024;
 constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
@@ -66,24 +83,34 @@ constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
 struct GemmArgs {
     int E, Mw, K, KB, MT, MTu, Mvalid;   // MTu: weight tiles per unit step (MT, or pairs)
-    int nmax, stages, tmem_cols;
+    int nmax, tmem_cols;
     const uint8_t* a_tiles;
     int ldo;
     void* out;
     const int32_t* counts;
     const int32_t* offsets;
-    const float* w_perm;       // routing weight of each permuted row (0 for pads)
+    const int32_t* sorted_ids;
+    int ktop;                  // assignments per token (flat index / ktop = token)
+    int A;                     // assignments (T * ktop): flat indices are below it
+    int capacity;              // rows of the permuted operands
+    const uint8_t* gather_src; // gate/up: token-order rows of K elements
+    long long src_row_bytes;
+    const float* w;            // down: routing weight of flat index f
     const float* w_scales;
     const uint32_t* act_amax;
     uint32_t* out_amax;
+    float* acc_zero;           // gate/up: fp32 buffer zeroed for a later reduction
+    long long acc_zero_vec4;   // its size in float4
     float* partials;
     int32_t* counters;
     int32_t* status;
+    int sched_after_wait;      // counts/offsets are the previous kernel's output
 };
 
 struct Ctl {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
+    uint64_t gfull[kMaxStages];   // gathered rows of a stage landed (this CTA)
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -110,6 +137,11 @@ struct Seg {
 };
 
 constexpr int kDynSmemMax = kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024;
+
+template <bool PAIR>
+__host__ __device__ constexpr int stages_for() { return PAIR ? 3 : 2; }
+template <bool PAIR>
+__host__ __device__ constexpr int kps_for() { return PAIR ? 2 : 4; }
 
 __device__ __forceinline__ int find_expert(const int* prefix, int E, int u) {
     int lo = 0, hi = E - 1;
@@ -208,12 +240,17 @@ __device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
 // One 16-column chunk (16 tokens) of the accumulator rows this thread owns.
 // Epilogue warp w (4..11) owns TMEM lane quarter q = w % 4 (rows 32q..32q+31)
 // and every other chunk (half h = (w - 4) / 4).  `sw` is the FP8 dequant
-// factor of this row; `wreg` holds the routing weights of the unit's tokens,
-// token t in lane t/8, register t%8.
+// factor of this row; `wreg` / `treg` hold the routing weights / token
+// indices (-1 for pads) of the unit's tokens, token j in lane j/8, register
+// j%8.
+//   EPI 0: h = SiLU(gate) * up -> bf16 rows of h (permuted order)
+//   EPI 1: w * y -> bf16 rows of y_perm (permuted order)
+//   EPI 2: w * y added (fp32) into row `token` of the accumulator
 template <bool FP8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int m_own, int c0,
                                                float (&v)[16], float sw, const float (&wreg)[8],
-                                               uint8_t* staging, float& amax) {
+                                               const int (&treg)[8], uint8_t* staging,
+                                               float& amax) {
     const int ew = (threadIdx.x >> 5) - kEpiWarp0;
     const int q = (threadIdx.x >> 5) & 3;
     const int lane = threadIdx.x & 31;
@@ -243,7 +280,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
                                       static_cast<long>(row) * g.ldo + col) = val;
         __syncwarp();
-    } else {
+    } else if constexpr (EPI == 1) {
         __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + ew * 1024);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -264,6 +301,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
             }
         }
         __syncwarp();
+    } else {
+        // lane = output column: each warp-wide add covers 32 consecutive
+        // floats (one 128-byte line) of one token's accumulator row
+        const int hcol = m_own * kBM + 32 * q + lane;
+        float* acc = static_cast<float*>(g.out);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float wi = __shfl_sync(kFull, wreg[i & 7], (c0 + i) >> 3);
+            const int ti = __shfl_sync(kFull, treg[i & 7], (c0 + i) >> 3);
+            if (ti >= 0 && hcol < g.Mvalid)
+                red_add_f32(acc + static_cast<long>(ti) * g.ldo + hcol, v[i] * wi);
+        }
     }
 }
 
@@ -273,23 +322,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB128,
                         const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
+    constexpr bool GATHER = EPI == 0;
+    constexpr int S = stages_for<PAIR>();
+    // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
+    constexpr int KPS = kps_for<PAIR>();
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ Ctl ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    // stage = kps consecutive k-blocks: A kps*16 KB (one bulk copy), B kps
+    // stage = KPS consecutive k-blocks: A KPS*16 KB (one bulk copy), B KPS
     // slots of nmax rows x 128 B
-    // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
-    constexpr int KPS = PAIR ? 2 : 4;
     const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
     const int a_stage_bytes = KPS * kATileBytes;
     // a pair member holds half of each token tile
     const int b_kb_bytes = (PAIR ? g.nmax / 2 : g.nmax) * kRowBytes;
     const int b_stage_bytes = KPS * b_kb_bytes;
     uint8_t* smA = base;
-    uint8_t* smB = smA + g.stages * a_stage_bytes;
-    uint8_t* staging = smB + g.stages * b_stage_bytes;
+    uint8_t* smB = smA + S * a_stage_bytes;
+    uint8_t* staging = smB + S * b_stage_bytes;
+
+    if (g.sched_after_wait) pdl_wait();   // the counts come from the previous kernel
 
     // ---- schedule tables: per-expert counts, offsets, token tiles, unit prefix
     {
@@ -297,8 +350,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int units = 0;
         int key = 0x7fffffff;
         if (e < g.E) {
-            const int c = __ldcg(g.counts + e);
-            ctl.off[e] = __ldcg(g.offsets + e);
+            int c = __ldcg(g.counts + e);
+            const int o = __ldcg(g.offsets + e);
+            if constexpr (kDebugChecks) {
+                // the expert's rows, padded to 16, must lie inside the capacity
+                if (c < 0 || o < 0 || o + ((c + 15) & ~15) > g.capacity) {
+                    report(g.status, MOE_ERR_DEVICE);
+                    c = 0;
+                }
+            }
+            ctl.off[e] = o;
             int nf = c / g.nmax;
             const int r = c - nf * g.nmax;
             int n = (r + 15) & ~15;
@@ -320,9 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 31) ctl.scan_tmp[warp] = inc;
         if (threadIdx.x == 0) {
-            for (int i = 0; i < g.stages; ++i) {
-                mbar_init(&ctl.full[i], 1);
+            for (int i = 0; i < S; ++i) {
+                // gate/up: the producer's weight copies plus one forwarded
+                // arrival per CTA for the gathered rows
+                mbar_init(&ctl.full[i], GATHER ? 1 + (PAIR ? 2 : 1) : 1);
                 mbar_init(&ctl.empty[i], 1);
+                mbar_init(&ctl.gfull[i], kGatherLanes);
             }
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&ctl.tfull[i], 1);
@@ -337,11 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (warp == 0 && lane == 0) {
             if constexpr (PAIR) tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB128);
-            tma_prefetch_desc(&tmB64);
-            tma_prefetch_desc(&tmB16);
+            if constexpr (!GATHER) {
+                tma_prefetch_desc(&tmB128);
+                tma_prefetch_desc(&tmB64);
+                tma_prefetch_desc(&tmB16);
+            }
         }
-        if (warp == 2) {
+        if (warp == kFwdWarp) {
             if constexpr (PAIR) {
                 tmem_alloc_pair(&ctl.tmem_base, g.tmem_cols);
                 tmem_relinquish_pair();
@@ -368,9 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // rank of e's partial tile among all partial tiles (keys are distinct)
         if (key != 0x7fffffff) {
-            int rank = 0;
-            for (int i = 0; i < g.E; ++i) rank += ctl.key[i] < key ? 1 : 0;
-            ctl.part_expert[rank] = e;
+            int rank_e = 0;
+            for (int i = 0; i < g.E; ++i) rank_e += ctl.key[i] < key ? 1 : 0;
+            ctl.part_expert[rank_e] = e;
         }
         const int n_has = __popc(__ballot_sync(0xffffffffu, key != 0x7fffffff));
         __syncthreads();
@@ -406,10 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool active = sc.n_dp > 0 || in_sk;
     auto cursor = [&]() { return Cursor{0, sc.n_dp, cta, G, g.KB, sc.unit0, sc.ws, sc.we}; };
     const uint32_t tmem_base = ctl.tmem_base;
-    const int S = g.stages;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ copy producer
         // (both CTAs of a pair run it; their copies complete on the rank-0
         // CTA's barrier, which the rank-0 producer arms for both)
         if (lane == 0) {
@@ -417,11 +482,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int bk_elems = FP8 ? 128 : 64;
             const int mt_last = g.MT - 1;
             // A pair loads full KPS-tile boxes of weights; a single CTA loads
-            // exactly the stage's k-blocks.
+            // exactly the stage's k-blocks.  The gate/up kernel's token rows
+            // are not counted here: the gather warps deliver them.
             auto stage_bytes = [&](const Seg& sg, int nk) -> uint32_t {
-                const int rows = PAIR ? sg.Nm / 2 : sg.N;
-                const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
-                const uint32_t b = static_cast<uint32_t>(nk * (n64 * 64 + n16 * 16) * kRowBytes);
+                uint32_t b = 0;
+                if constexpr (!GATHER) {
+                    const int rows = PAIR ? sg.Nm / 2 : sg.N;
+                    const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
+                    b = static_cast<uint32_t>(nk * (n64 * 64 + n16 * 16) * kRowBytes);
+                }
                 return PAIR ? 2u * (static_cast<uint32_t>(KPS * kATileBytes) + b)
                             : static_cast<uint32_t>(nk * kATileBytes) + b;
             };
@@ -498,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (rank == 0) mbar_arrive_expect_tx(&ctl.full[st], stage_bytes(sg, nk));
                         load_a(sg, kb, nk, st);
                     }
-                    load_b(sg, kb, nk, st);
+                    if constexpr (!GATHER) load_b(sg, kb, nk, st);
                     if (++st == S) {
                         st = 0;
                         par ^= 1u;
@@ -509,6 +578,109 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl.prod_pos = it > static_cast<uint32_t>(early) ? it : static_cast<uint32_t>(early);
         }
         __syncwarp();
+    } else if (warp >= kGatherWarp0) {
+        // ------------------------------------------------ gather (gate/up)
+        // Lane gl copies 16-byte chunk c = gl % 8 of rows r0 + 16 i (r0 =
+        // gl / 8) of this CTA's token rows, for every k-block of a stage: a
+        // warp covers four whole 128-byte row segments per instruction.  In
+        // the 128-byte swizzle, chunk c of row r sits at c ^ (r % 8), which is
+        // fixed per lane.  Pads (sorted_ids = -1), rows past the tile and
+        // bytes past the end of a row are zero-filled.
+        if constexpr (GATHER) {
+            const int gl = threadIdx.x - kGatherWarp0 * 32;
+            const int c = gl & 7, r0 = gl >> 3;
+            const uint32_t cs = static_cast<uint32_t>((c ^ (r0 & 7)) << 4);
+            constexpr int kMaxRowIters = 128 / kGatherRowsPerPass;   // 8
+            const uint32_t smB_u32 = smem_u32(smB);
+            pdl_wait();   // sorted_ids and the source rows come from earlier kernels
+            int st = 0;
+            uint32_t par = 1;
+            Cursor cur = cursor();
+            int u, kb0, kb1;
+            bool ok = true;
+            while (ok && active && cur.next(u, kb0, kb1)) {
+                const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
+                const int rows = PAIR ? sg.Nm / 2 : sg.N;
+                const int first = rank * rows;     // this CTA's first row of the tile
+                long long src_off[kMaxRowIters];
+#pragma unroll
+                for (int i = 0; i < kMaxRowIters; ++i) {
+                    const int r = r0 + kGatherRowsPerPass * i;
+                    int sid = -1;
+                    if (r < rows && first + r < sg.N) sid = __ldg(g.sorted_ids + sg.b_row + first + r);
+                    if constexpr (kDebugChecks) {
+                        if (sid < -1 || sid >= g.A) {
+                            report(g.status, MOE_ERR_DEVICE);
+                            sid = -1;
+                        }
+                    }
+                    src_off[i] = sid >= 0 ? static_cast<long long>(sid / g.ktop) * g.src_row_bytes
+                                          : -1;
+                }
+                for (int kb = sg.kb0; kb < sg.kb1; kb += KPS) {
+                    const int nk = min(KPS, sg.kb1 - kb);
+                    if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
+                        raise_abort(ctl, g.status);
+                        ok = false;
+                        break;
+                    }
+                    for (int q = 0; q < nk; ++q) {
+                        const long long kofs = static_cast<long long>(kb + q) * kRowBytes + c * 16;
+                        const bool in_row = kofs < g.src_row_bytes;
+                        const uint32_t dst0 = smB_u32 + st * b_stage_bytes + q * b_kb_bytes + cs;
+#pragma unroll
+                        for (int i = 0; i < kMaxRowIters; ++i) {
+                            const int r = r0 + kGatherRowsPerPass * i;
+                            if (r < rows) {
+                                const bool v = in_row && src_off[i] >= 0;
+                                const uint8_t* src = v ? g.gather_src + src_off[i] + kofs
+                                                       : g.gather_src;
+                                cp_async16(dst0 + r * kRowBytes, src, v ? 16u : 0u);
+                            }
+                        }
+                    }
+                    cp_async_arrive_noinc(&ctl.gfull[st]);
+                    if (++st == S) {
+                        st = 0;
+                        par ^= 1u;
+                    }
+                }
+            }
+            // no copy may still target shared memory when the CTA moves on
+            cp_async_wait_all();
+        }
+    } else if (warp == kFwdWarp) {
+        // ------------------------------------------------ gather forwarder
+        // Waits until a stage's gathered rows have landed in this CTA's
+        // shared memory, makes them visible to the async proxy (the tensor
+        // core reads operands through it) and arrives on the MMA issuer's
+        // barrier (the rank-0 CTA's, for a pair).
+        if constexpr (GATHER) {
+            if (lane == 0) {
+                int st = 0;
+                uint32_t ph = 0;
+                Cursor cur = cursor();
+                int u, kb0, kb1;
+                bool ok = true;
+                while (ok && active && cur.next(u, kb0, kb1)) {
+                    for (int kb = kb0; kb < kb1; kb += KPS) {
+                        if (!mbar_wait(&ctl.gfull[st], ph, &ctl.abort)) {
+                            raise_abort(ctl, g.status);
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_smem();
+                        if constexpr (PAIR) mbar_arrive_cluster(leader_addr(&ctl.full[st]));
+                        else mbar_arrive_cluster(smem_u32(&ctl.full[st]));
+                        if (++st == S) {
+                            st = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+        }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && active && rank == 0) {
@@ -540,7 +712,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = make_idesc<FP8>(PAIR ? 2 * kBM : kBM, s.Nm);
                 for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
                     const int nk = s.kb1 - kb;
-                    if (!mbar_wait(&ctl.full[st], ph, &ctl.abort)) {
+                    // gathered rows arrive through a release at cluster scope
+                    const bool got = GATHER ? mbar_wait_cluster(&ctl.full[st], ph, &ctl.abort)
+                                            : mbar_wait(&ctl.full[st], ph, &ctl.abort);
+                    if (!got) {
                         raise_abort(ctl, g.status);
                         ok = false;
                         break;
@@ -581,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl.mma_pos = it;
         }
         __syncwarp();
-    } else if (warp >= kEpiWarp0) {
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiThreads / 32) {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;                     // TMEM lane quarter
         const int half = (warp - kEpiWarp0) >> 2;   // which chunks: c0 = 16*(2j + half)
@@ -596,6 +771,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else mbar_arrive(&ctl.tempty[acc]);
             }
         };
+        // the scales and the routing outputs come from earlier kernels
+        pdl_wait();
+        if constexpr (EPI == 0) {
+            // zero this CTA's slice of the fp32 buffer a later down kernel
+            // reduces into (its kernel starts only after this one completes)
+            if (g.acc_zero) {
+                const long long nthreads = static_cast<long long>(gridDim.x) * kEpiThreads;
+                const long long tid = static_cast<long long>(blockIdx.x) * kEpiThreads +
+                                      (threadIdx.x - kEpiWarp0 * 32);
+                float4* z = reinterpret_cast<float4*>(g.acc_zero);
+                for (long long i = tid; i < g.acc_zero_vec4; i += nthreads)
+                    z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
         float act_scale = 1.0f;
         if constexpr (FP8) act_scale = fp8_scale_from_amax(__ldcg(g.act_amax));
         float amax = 0.0f;
@@ -606,20 +795,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Seg s = make_seg<PAIR>(ctl, g, u, kb0, kb1);
             const int acc = si & 1;
             const int m_own = PAIR ? 2 * s.m + rank : s.m;   // this CTA's 128-row weight tile
-            // per-unit constants: FP8 dequant factor of this row, routing weights
+            // per-unit constants: FP8 dequant factor of this row, routing
+            // weights and token indices of the unit's tokens
             float sw = 1.0f;
             if constexpr (FP8)
-                sw = act_scale * __ldg(g.w_scales + s.e * 3 + (EPI == 1 ? 2 : (lane < 16 ? 0 : 1)));
+                sw = act_scale * __ldg(g.w_scales + s.e * 3 + (EPI != 0 ? 2 : (lane < 16 ? 0 : 1)));
             float wreg[8];
-            if constexpr (EPI == 1) {
-                if (8 * lane < s.N) {
-                    const float4* wp = reinterpret_cast<const float4*>(g.w_perm + s.b_row + 8 * lane);
-                    const float4 a = __ldcg(wp), b = __ldcg(wp + 1);
-                    wreg[0] = a.x; wreg[1] = a.y; wreg[2] = a.z; wreg[3] = a.w;
-                    wreg[4] = b.x; wreg[5] = b.y; wreg[6] = b.z; wreg[7] = b.w;
-                } else {
+            int treg[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) wreg[i] = 0.0f;
+            for (int i = 0; i < 8; ++i) {
+                wreg[i] = 0.0f;
+                treg[i] = -1;
+            }
+            if constexpr (EPI != 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int j = 8 * lane + i;
+                    if (j < s.N) {
+                        int sid = __ldg(g.sorted_ids + s.b_row + j);
+                        if constexpr (kDebugChecks) {
+                            if (sid < -1 || sid >= g.A) {
+                                report(g.status, MOE_ERR_DEVICE);
+                                sid = -1;
+                            }
+                        }
+                        if (sid >= 0) {
+                            wreg[i] = __ldg(g.w + sid);
+                            treg[i] = sid / g.ktop;
+                        }
+                    }
                 }
             }
             if (!mbar_wait(&ctl.tfull[acc], (si >> 1) & 1u, &ctl.abort)) {
@@ -632,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
                     float v[16];
                     tmem_ld16(taddr + c0, v);
-                    epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, staging, amax);
+                    epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, treg, staging, amax);
                 }
                 release(acc);
             } else {
@@ -674,7 +878,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] += ld_cg(p + i * kBM);
                         }
-                        epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, staging, amax);
+                        epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, treg, staging,
+                                                 amax);
                     }
                     if (threadIdx.x == kEpiWarp0 * 32) g.counters[ctr] = 0;
                 }
@@ -706,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // neither CTA of a pair frees its TMEM before the pair's MMAs, copies
     // and epilogues are all done
     if constexpr (PAIR) cluster_sync();
-    if (warp == 2) {
+    if (warp == kFwdWarp) {
         tc_fence_after();
         if constexpr (PAIR) tmem_dealloc_pair(tmem_base, g.tmem_cols);
         else tmem_dealloc(tmem_base, g.tmem_cols);
@@ -814,6 +1019,17 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b128, const CUtens
     return cudaLaunchKernelEx(&cfg, kern, a, b128, b64, b16, g);
 }
 
+template <bool FP8, bool PAIR>
+cudaError_t launch_epi(int epi, const CUtensorMap& a, const CUtensorMap& b128,
+                       const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& g, int grid,
+                       int smem, cudaStream_t s) {
+    switch (epi) {
+        case 0: return launch_t<FP8, 0, PAIR>(a, b128, b64, b16, g, grid, smem, s);
+        case 1: return launch_t<FP8, 1, PAIR>(a, b128, b64, b16, g, grid, smem, s);
+        default: return launch_t<FP8, 2, PAIR>(a, b128, b64, b16, g, grid, smem, s);
+    }
+}
+
 int pow2_at_least(int v) {
     int p = 32;
     while (p < v) p <<= 1;
@@ -831,10 +1047,15 @@ int device_sm_count() {
 
 int gemm_nmax_for(int T, int k, int E) {
     // Twice the mean tokens per expert, in steps of 16 (16..256); experts with
-    // more tokens are split into several token tiles.
+    // more tokens are split into several token tiles.  Above 64 the tiles run
+    // on CTA pairs, whose MMA N is a multiple of 32 (16 token rows per CTA),
+    // so the cap is rounded to 32: every tile's MMA N then fits both the
+    // per-k-block operand slot (nmax/2 rows per CTA) and the accumulator
+    // stride (nmax columns).
     const long mean2 = (2L * T * k + E - 1) / E;
     long n = (mean2 + 15) & ~15L;
     if (n < 16) n = 16;
+    if (n > 64) n = (n + 31) & ~31L;
     if (n > 256) n = 256;
     return static_cast<int>(n);
 }
@@ -857,53 +1078,61 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     const bool pair = p.nmax > 64;
     g.MTu = pair ? (p.MT + 1) / 2 : p.MT;
     g.a_tiles = static_cast<const uint8_t*>(p.weights);
-    // Two stages of several k-blocks each: small token tiles (weight
-    // streaming) take 4 k-blocks (64 KB weight copies), large ones 2 (32 KB
-    // weights + 64 KB activations).  Measured on B200: fewer, larger copies
-    // sustain more bandwidth than many 16 KB stages, for both regimes.
-    const int kps = pair ? 2 : 4;   // the kernel's KPS
-    const int max_stages = pair ? 3 : 2;
+    // Stages of several k-blocks each: small token tiles (weight streaming)
+    // take 2 stages of 4 k-blocks (64 KB weight copies), large ones 3 stages
+    // of 2 (32 KB weights + 32 KB activations per CTA).  Measured on B200:
+    // fewer, larger copies sustain more bandwidth than many 16 KB stages, for
+    // both regimes.
+    const int kps = pair ? kps_for<true>() : kps_for<false>();
+    const int stages = pair ? stages_for<true>() : stages_for<false>();
     const int stage_bytes = kps * (kATileBytes + (pair ? p.nmax / 2 : p.nmax) * kRowBytes);
-    int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
-    if (stages > max_stages) stages = max_stages;
-    if (stages < 2) return cudaErrorInvalidValue;
-    g.stages = stages;
+    const int smem = 1024 + stages * stage_bytes + kStagingBytes;
+    if (smem > kDynSmemMax) return cudaErrorInvalidValue;
     g.tmem_cols = pow2_at_least(2 * p.nmax);
     g.ldo = p.ldo;
     g.out = p.out;
     g.counts = p.counts;
     g.offsets = p.offsets;
-    g.w_perm = p.w_perm;
+    g.sorted_ids = p.sorted_ids;
+    g.ktop = p.ktop;
+    g.A = p.A;
+    g.capacity = p.capacity;
+    g.gather_src = static_cast<const uint8_t*>(p.gather_src);
+    g.src_row_bytes = static_cast<long long>(p.K) * (p.fp8 ? 1 : 2);
+    g.w = p.w;
     g.w_scales = p.w_scales;
     g.act_amax = p.act_amax;
     g.out_amax = p.out_amax;
+    g.acc_zero = p.acc_zero;
+    g.acc_zero_vec4 = static_cast<long long>(p.acc_zero_floats / 4);
     g.partials = p.partials;
     g.counters = p.counters;
     g.status = p.status;
+    g.sched_after_wait = p.sched_after_wait ? 1 : 0;
+    if (p.epi == 0 && (!p.gather_src || !p.sorted_ids || p.ktop < 1)) return cudaErrorInvalidValue;
+    if (p.epi != 0 && (!p.sorted_ids || !p.w)) return cudaErrorInvalidValue;
+    if (p.acc_zero_floats % 4 != 0) return cudaErrorInvalidValue;
     CUtensorMap ta, tb128, tb64, tb16;
     memset(&ta, 0, sizeof(ta));
-    if (!make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
-        !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
-        !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16))
+    memset(&tb128, 0, sizeof(tb128));
+    memset(&tb64, 0, sizeof(tb64));
+    memset(&tb16, 0, sizeof(tb16));
+    // the down kernel's activation rows (h, permuted order) come by TMA; the
+    // gate/up kernel gathers its rows and uses no activation maps
+    if (p.epi != 0 && (!make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
+                       !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
+                       !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16)))
         return cudaErrorInvalidValue;
     if (pair && !make_tile_map(&ta, p.weights, static_cast<long>(p.E) * p.MT * p.KB, kps))
         return cudaErrorInvalidValue;
     int grid = device_sm_count();
     if (p.max_ctas > 0 && p.max_ctas < grid) grid = p.max_ctas;
     if (pair) grid = grid < 2 ? 2 : grid & ~1;
-    const int smem = 1024 + stages * stage_bytes + kStagingBytes;
-    if (pair) {
-        if (p.fp8)
-            return p.epi == 0 ? launch_t<true, 0, true>(ta, tb128, tb64, tb16, g, grid, smem, s)
-                              : launch_t<true, 1, true>(ta, tb128, tb64, tb16, g, grid, smem, s);
-        return p.epi == 0 ? launch_t<false, 0, true>(ta, tb128, tb64, tb16, g, grid, smem, s)
-                          : launch_t<false, 1, true>(ta, tb128, tb64, tb16, g, grid, smem, s);
-    }
-    if (p.fp8)
-        return p.epi == 0 ? launch_t<true, 0, false>(ta, tb128, tb64, tb16, g, grid, smem, s)
-                          : launch_t<true, 1, false>(ta, tb128, tb64, tb16, g, grid, smem, s);
-    return p.epi == 0 ? launch_t<false, 0, false>(ta, tb128, tb64, tb16, g, grid, smem, s)
-                      : launch_t<false, 1, false>(ta, tb128, tb64, tb16, g, grid, smem, s);
+    if (pair)
+        return p.fp8 ? launch_epi<true, true>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s)
+                     : launch_epi<false, true>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s);
+    return p.fp8 ? launch_epi<true, false>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s)
+                 : launch_epi<false, false>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s);
 }
 
 }  // namespace moe

@@ -69,10 +69,10 @@ cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
                                        cudaStream_t s, int32_t* ctl = nullptr, int ctl_ints = 0,
                                        const void* x = nullptr, long x_elems = 0,
-                                       uint32_t* amax_out = nullptr);
-// Batches small enough for the single-CTA kernel to also take amax(x) (FP8):
-// up to 64 KB of x (measured on B200: at 184 KB the one CTA took longer than
-// the separate amax kernel it replaced).
+                                       uint32_t* amax_out = nullptr, void* xq_out = nullptr);
+// Batches small enough for the single-CTA kernel to also take amax(x) and
+// quantise x (FP8): up to 64 KB of x (measured on B200: at 184 KB the one CTA
+// took longer than the separate amax kernel it replaced).
 constexpr long kSmallAmaxElems = 32768;
 cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int block_m,
                                  int capacity, int32_t* counts, int32_t* offsets,
@@ -81,19 +81,20 @@ cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int bl
                                  cudaStream_t s);
 
 // ---- a3/a5/a7 and packing (elementwise.cu)
-// The gathers also write w_perm[p] = w[sorted_ids[p]] (0 for pads).
-cudaError_t launch_gather_bf16(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                               int E, int k, int H, int capacity, const float* w, void* x_perm,
-                               float* w_perm, cudaStream_t s);
 cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaStream_t s);
-cudaError_t launch_gather_fp8(const void* x, const int32_t* sorted_ids, const int32_t* offsets,
-                              int E, int k, int H, int capacity, const uint32_t* amax_bits,
-                              const float* w, void* x_perm, float* w_perm, cudaStream_t s);
+// FP8 x in token order: xq = RNE_sat(x * (1 / s_x)), s_x from amax_bits.
+cudaError_t launch_quant_x_fp8(const void* x, long n, const uint32_t* amax_bits, void* xq,
+                               cudaStream_t s);
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
                                   int capacity, const uint32_t* amax_bits, void* h_q,
                                   cudaStream_t s);
+// rows: rows of y_perm (debug builds check inv_perm against it; INT32_MAX if
+// unknown), status: where such a fault is reported (may be null)
 cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, int T, int k, int H,
-                           void* out, cudaStream_t s);
+                           void* out, cudaStream_t s, int rows = 0x7fffffff,
+                           int32_t* status = nullptr);
+// out (bf16) = acc (fp32), n elements (n % 8 == 0)
+cudaError_t launch_finalize(const float* acc, long n, void* out, cudaStream_t s);
 cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, const void* Wu,
                                 const void* Wd, void* packed, float* scales, uint32_t* amax_tmp,
                                 cudaStream_t s);
@@ -102,26 +103,35 @@ cudaError_t launch_wait_timeout_selftest(int32_t* status, int timeout_us, cudaSt
 // ---- a4/a6 (grouped_gemm.cu)
 struct GemmProblem {
     int fp8;              // 0 bf16, 1 e4m3
-    int epi;              // 0: gate/up -> SiLU*up -> h; 1: down -> * w -> y
+    int epi;              // 0: gate/up, rows gathered from gather_src -> SiLU*up -> h
+                          // 1: down -> * w -> bf16 rows of out (permuted order)
+                          // 2: down -> * w -> added into fp32 row `token` of out
     int E, Mw, K;         // weight rows per expert, reduction length
     int Mvalid;           // weight rows per expert that are real (masking)
     int nmax;             // token-tile cap (multiple of 16, <= 256)
-    int capacity;         // rows of the activation operand
+    int capacity;         // rows of the permuted operands
     const void* weights;  // packed tiles of this matrix (see PackedGeom)
     int MT, KB;           // row tiles and k-blocks per expert
-    const void* act;      // [capacity, K]
-    void* out;            // [capacity, ldo] bf16
+    const void* act;      // epi 1/2: [capacity, K] rows in permuted order
+    const void* gather_src;  // epi 0: [T, K] rows in token order
+    void* out;            // epi 0/1: [capacity, ldo] bf16; epi 2: [T, ldo] f32
     int ldo;
     const int32_t* counts;
     const int32_t* offsets;
-    const float* w_perm;         // epi 1: routing weight per permuted row
+    const int32_t* sorted_ids;
+    int ktop;                    // k (flat assignment index / k = token)
+    int A;                       // T * k
+    const float* w;              // epi 1/2: routing weight by flat index [T*k]
     const float* w_scales;       // [E][3] (FP8)
     const uint32_t* act_amax;    // FP8: amax bits of the activation operand
     uint32_t* out_amax;          // FP8 epi 0: amax of h (bits)
+    float* acc_zero;             // epi 0: fp32 buffer to zero (may be null)
+    long acc_zero_floats;        // its length, a multiple of 4
     float* partials;             // [max_ctas][2][128*nmax] f32
     int32_t* counters;           // [max_ctas] zeroed
     int32_t* status;
     int max_ctas;
+    int sched_after_wait;        // counts/offsets are written by the previous kernel
 };
 int gemm_nmax_for(int T, int k, int E);
 size_t gemm_partials_bytes(int nmax);

@@ -2,6 +2,8 @@
 // validation (nothing is launched on a bad argument), workspace carving, and
 // the order of launches on the caller's stream.  Never allocates, never
 // synchronises (except moe_check_status, whose job is to read the device).
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdint>
 #include <cstring>
 
@@ -58,30 +60,35 @@ struct Carver {
 
 struct FfnBuffers {
     int32_t* ctl;
-    float* w_perm;
-    void* x_perm;
+    void* xq;         // FP8: e4m3 codes of x, token order [T, H]
     void* h;
     void* h_q;
     float* partials;
 };
 
-void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int cap, int H, int I, int nmax) {
-    const size_t elt = dt == MOE_FP8_E4M3 ? 1 : 2;
-    b.w_perm = c.take<float>(sizeof(float) * static_cast<size_t>(cap > 0 ? cap : 1));
-    b.x_perm = c.take<void>(static_cast<size_t>(cap) * H * elt);
+void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int T, int cap, int H, int I,
+                    int nmax) {
+    const bool fp8 = dt == MOE_FP8_E4M3;
+    b.xq = fp8 ? c.take<void>(static_cast<size_t>(T) * H) : nullptr;
     b.h = c.take<void>(static_cast<size_t>(cap) * I * 2);
-    b.h_q = dt == MOE_FP8_E4M3 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
+    b.h_q = fp8 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
     b.partials = c.take<float>(gemm_partials_bytes(nmax));
 }
 
 // The control block is carved first, so a missing caller status word means
 // the first int32 of the workspace.
-FfnBuffers carve_ffn(Carver& c, moe_dtype dt, int cap, int H, int I, int nmax) {
+FfnBuffers carve_ffn(Carver& c, moe_dtype dt, int T, int cap, int H, int I, int nmax) {
     FfnBuffers b;
     b.ctl = c.take<int32_t>(sizeof(int32_t) * kCtlInts);
-    carve_ffn_rest(c, b, dt, cap, H, I, nmax);
+    carve_ffn_rest(c, b, dt, T, cap, H, I, nmax);
     return b;
 }
+
+// How a forward call forms out[t] = sum_j y(t, j).
+enum class Combine {
+    kGatherSum,   // y_perm rows written by the down GEMM, summed in fixed j order
+    kFused        // the down GEMM's epilogue adds w*y into an fp32 accumulator
+};
 
 struct FfnCall {
     moe_dtype dt;
@@ -93,15 +100,26 @@ struct FfnCall {
     const int32_t* sorted_ids;
     const void* packed;
     const float* scales;
-    void* y_perm;
+    void* y_out;                 // y_perm [cap, H] bf16, or the fp32 accumulator [T, H]
     int32_t* status;
     int max_ctas;
-    bool x_amax_ready = false;   // amax(x) already in the control block (FP8)
+    bool x_ready = false;        // FP8: amax(x) and the codes of x already written
+    bool counts_from_prev = false;  // the permutation is the previous kernel's output
+    Combine combine = Combine::kGatherSum;
 };
 
 void record(moe_event_t* ev, int i, cudaStream_t s) {
     if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s);
 }
+
+// NVTX range over the host-side launches of one stage (shown by profilers
+// such as Nsight Systems / Compute; free when no tool is attached).
+struct Range {
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range&) = delete;
+    Range& operator=(const Range&) = delete;
+};
 
 // a3..a6 on carved buffers.  The control block must already be zeroed.
 moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaStream_t s) {
@@ -109,21 +127,20 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     const int nmax = gemm_nmax_for(f.T, f.k, f.E);
     uint32_t* amax_x = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxX);
     uint32_t* amax_h = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxH);
-    cudaError_t e;
-    if (fp8) {
-        e = f.x_amax_ready ? cudaSuccess
-                           : launch_amax_bf16(f.x, static_cast<long>(f.T) * f.H, amax_x, s);
-        if (e == cudaSuccess)
-            e = launch_gather_fp8(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, amax_x,
-                                  f.w, b.x_perm, b.w_perm, s);
-    } else {
-        e = launch_gather_bf16(f.x, f.sorted_ids, f.offsets, f.E, f.k, f.H, f.cap, f.w, b.x_perm,
-                               b.w_perm, s);
+    const long x_elems = static_cast<long>(f.T) * f.H;
+    bool counts_from_prev = f.counts_from_prev;
+    if (fp8 && !f.x_ready) {
+        // a3 (FP8): amax(x) and the e4m3 codes of x, in token order
+        Range r("moe: x quantisation (a3)");
+        if (launch_amax_bf16(f.x, x_elems, amax_x, s) != cudaSuccess ||
+            launch_quant_x_fp8(f.x, x_elems, amax_x, b.xq, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        counts_from_prev = false;
     }
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 2, s);
 
     const PackedGeom geo = packed_geom(fp8, f.E, f.H, f.I);
+    const bool fused = f.combine == Combine::kFused;
     GemmProblem gu{};
     gu.fp8 = fp8;
     gu.epi = 0;
@@ -136,28 +153,40 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     gu.weights = f.packed;
     gu.MT = geo.mt_gu;
     gu.KB = geo.kb_gu;
-    gu.act = b.x_perm;
+    gu.gather_src = fp8 ? b.xq : f.x;
     gu.out = b.h;
     gu.ldo = f.I;
     gu.counts = f.counts;
     gu.offsets = f.offsets;
+    gu.sorted_ids = f.sorted_ids;
+    gu.ktop = f.k;
+    gu.A = f.T * f.k;
     gu.w_scales = f.scales;
     gu.act_amax = amax_x;
     gu.out_amax = amax_h;
+    gu.acc_zero = fused ? static_cast<float*>(f.y_out) : nullptr;
+    gu.acc_zero_floats = fused ? x_elems : 0;
     gu.partials = b.partials;
     gu.counters = b.ctl + kCtlCountersGu;
     gu.status = f.status;
     gu.max_ctas = f.max_ctas;
-    if (launch_grouped_gemm(gu, s) != cudaSuccess) return MOE_ERR_CUDA;
+    gu.sched_after_wait = counts_from_prev ? 1 : 0;
+    {
+        Range r("moe: gate/up GEMM (a3 gather + a4)");
+        if (launch_grouped_gemm(gu, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     record(ev, 3, s);
 
-    if (fp8 && launch_quant_rows_fp8(b.h, f.offsets, f.E, f.I, f.cap, amax_h, b.h_q, s) !=
-                   cudaSuccess)
-        return MOE_ERR_CUDA;
+    if (fp8) {
+        Range r("moe: h quantisation (a5)");
+        if (launch_quant_rows_fp8(b.h, f.offsets, f.E, f.I, f.cap, amax_h, b.h_q, s) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
     record(ev, 4, s);
 
     GemmProblem dn = gu;
-    dn.epi = 1;
+    dn.epi = fused ? 2 : 1;
     dn.Mw = f.H;
     dn.K = f.I;
     dn.Mvalid = f.H;
@@ -165,13 +194,20 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     dn.MT = geo.mt_dn;
     dn.KB = geo.kb_dn;
     dn.act = fp8 ? b.h_q : b.h;
-    dn.out = f.y_perm;
+    dn.gather_src = nullptr;
+    dn.out = f.y_out;
     dn.ldo = f.H;
-    dn.w_perm = b.w_perm;
+    dn.w = f.w;
     dn.act_amax = amax_h;
     dn.out_amax = nullptr;
+    dn.acc_zero = nullptr;
+    dn.acc_zero_floats = 0;
     dn.counters = b.ctl + kCtlCountersDn;
-    if (launch_grouped_gemm(dn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    dn.sched_after_wait = 0;   // the permutation is at least two kernels back
+    {
+        Range r(fused ? "moe: down GEMM + combine (a6 + a7)" : "moe: down GEMM (a6)");
+        if (launch_grouped_gemm(dn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     record(ev, 5, s);
     return MOE_OK;
 }
@@ -179,7 +215,7 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
 size_t ffn_ws_bytes(moe_dtype dt, int T, int k, int E, int H, int I, int block_m) {
     Carver c{nullptr};
     const int cap = moe_permute_capacity(T, k, E, block_m);
-    carve_ffn(c, dt, cap, H, I, gemm_nmax_for(T, k, E));
+    carve_ffn(c, dt, T, cap, H, I, gemm_nmax_for(T, k, E));
     return c.used;
 }
 
@@ -193,7 +229,7 @@ struct FwdBuffers {
     int32_t* inv_perm;
     int32_t* tiles;
     int32_t* chunk_counts;
-    void* y_perm;
+    void* y_out;      // y_perm (bf16 [cap, H]) or the fp32 accumulator [T, H]
     FfnBuffers ffn;
 };
 
@@ -211,9 +247,25 @@ FwdBuffers carve_fwd(Carver& c, moe_dtype dt, int T, int k, int E, int H, int I,
     b.inv_perm = c.take<int32_t>(sizeof(int32_t) * (A > 0 ? A : 1));
     b.tiles = c.take<int32_t>(sizeof(int32_t) * (cap / block_m + 1));
     b.chunk_counts = c.take<int32_t>(sizeof(int32_t) * permute_chunks(A) * E);
-    b.y_perm = c.take<void>(static_cast<size_t>(cap) * H * 2);
-    carve_ffn_rest(c, b.ffn, dt, cap, H, I, gemm_nmax_for(T, k, E));
+    // one region serves either combine: y_perm or the fp32 accumulator
+    const size_t yperm = static_cast<size_t>(cap) * H * 2;
+    const size_t acc = static_cast<size_t>(T) * H * 4;
+    b.y_out = c.take<void>(yperm > acc ? yperm : acc);
+    carve_ffn_rest(c, b.ffn, dt, T, cap, H, I, gemm_nmax_for(T, k, E));
     return b;
+}
+
+// The combine a forward call uses.  The gather-sum is deterministic (a fixed
+// summation order); the fused reduction skips the y_perm round trip through
+// memory but adds in arrival order.  Auto picks the fused form where y_perm
+// is large.
+constexpr long kFusedMinAssignments = 4096;
+
+Combine pick_combine(int mode, int T, int k) {
+    if (mode == MOE_COMBINE_DETERMINISTIC) return Combine::kGatherSum;
+    if (mode == MOE_COMBINE_FUSED) return Combine::kFused;
+    return static_cast<long>(T) * k >= kFusedMinAssignments ? Combine::kFused
+                                                           : Combine::kGatherSum;
 }
 
 }  // namespace
@@ -325,12 +377,14 @@ moe_status moe_grouped_ffn(const moe_ffn_args* a, void* ws, size_t ws_bytes, moe
     if (!ws || ws_bytes < need_ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     Carver c{static_cast<char*>(ws)};
-    const FfnBuffers b = carve_ffn(c, a->dtype, a->capacity, a->H, a->I, gemm_nmax_for(a->T, a->k, a->E));
+    const FfnBuffers b = carve_ffn(c, a->dtype, a->T, a->capacity, a->H, a->I,
+                                   gemm_nmax_for(a->T, a->k, a->E));
     if (cudaMemsetAsync(b.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, a->capacity, a->x, a->w, a->counts,
               a->offsets, a->sorted_ids, a->packed, a->scales, a->y_perm,
               a->status ? a->status : b.ctl + kCtlStatus, a->max_ctas};
+    f.counts_from_prev = true;   // made by the caller's earlier calls: read after the wait
     return run_ffn(f, b, nullptr, s);
 }
 
@@ -360,6 +414,8 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     if (st != MOE_OK) return st;
     if (a->events && a->n_events != 7) return MOE_ERR_INVALID_ARG;
     if (a->max_ctas < 0) return MOE_ERR_INVALID_ARG;
+    if (a->combine < MOE_COMBINE_AUTO || a->combine > MOE_COMBINE_FUSED)
+        return MOE_ERR_INVALID_ARG;
     if (a->T == 0) return MOE_OK;
     if (!a->x || !a->logits || !a->packed || !a->out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(a->x) || !aligned16(a->packed) || !aligned16(a->out))
@@ -384,14 +440,21 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     // kernels are done with it.
     cudaError_t e;
     const long x_elems = static_cast<long>(a->T) * a->H;
+    const long A = static_cast<long>(a->T) * a->k;
+    const bool fp8 = a->dtype == MOE_FP8_E4M3;
     const bool small = fused_route_permute_ok(a->T, a->k);
-    const bool amax_fused = small && a->dtype == MOE_FP8_E4M3 && x_elems <= kSmallAmaxElems;
+    // FP8 with a small x: the single-CTA route kernel also takes amax(x) and
+    // writes the codes of x
+    const bool x_fused = small && fp8 && x_elems <= kSmallAmaxElems;
+    Range whole("moe_forward");
+    nvtxRangePushA("moe: route + permute (a1, a2)");
     if (small) {
         e = launch_route_permute_small(
             a->logits, a->T, a->E, a->k, block_m, cap, ids, w, b.counts, b.offsets, b.sorted_ids,
             b.inv_perm, b.tiles, b.num_tiles, status, s, b.ffn.ctl, kCtlInts,
-            amax_fused ? a->x : nullptr, x_elems,
-            amax_fused ? reinterpret_cast<uint32_t*>(b.ffn.ctl + kCtlAmaxX) : nullptr);
+            x_fused ? a->x : nullptr, x_elems,
+            x_fused ? reinterpret_cast<uint32_t*>(b.ffn.ctl + kCtlAmaxX) : nullptr,
+            x_fused ? b.ffn.xq : nullptr);
     } else {
         e = launch_route_topk(a->logits, a->T, a->E, a->k, ids, w, s, b.ffn.ctl, kCtlInts);
         if (e == cudaSuccess)
@@ -399,14 +462,25 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
                                      b.sorted_ids, b.inv_perm, b.tiles, b.num_tiles,
                                      b.chunk_counts, status, s);
     }
+    nvtxRangePop();
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 1, s);
     FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, cap, a->x, w, b.counts, b.offsets,
-              b.sorted_ids, a->packed, a->scales, b.y_perm, status, a->max_ctas, amax_fused};
+              b.sorted_ids, a->packed, a->scales, b.y_out, status, a->max_ctas};
+    f.x_ready = x_fused;
+    // the single-CTA permutation (the only one for A <= 2048) is the kernel
+    // right before the gate/up GEMM, unless FP8 kernels come between
+    f.counts_from_prev = permute_chunks(A) <= 1;
+    f.combine = pick_combine(a->combine, a->T, a->k);
     st = run_ffn(f, b.ffn, ev, s);
     if (st != MOE_OK) return st;
-    if (launch_combine(b.y_perm, b.inv_perm, a->T, a->k, a->H, a->out, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    {
+        Range r("moe: combine (a7)");
+        e = f.combine == Combine::kFused
+                ? launch_finalize(static_cast<const float*>(b.y_out), x_elems, a->out, s)
+                : launch_combine(b.y_out, b.inv_perm, a->T, a->k, a->H, a->out, s, cap, status);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     record(ev, 6, s);
     return MOE_OK;
 }

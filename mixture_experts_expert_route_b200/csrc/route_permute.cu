@@ -37,17 +37,6 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kPermChunk = 512;
 constexpr int kScanBatch = 16;
 
-// Largest |value| of 8 packed bf16.
-__device__ __forceinline__ float amax8(uint4 v) {
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(u[i] << 16)),
-                           fabsf(__uint_as_float(u[i] & 0xffff0000u))));
-    return m;
-}
-
 // Selection order as one 64-bit key, larger first: an order-preserving map of
 // the logit (-0 folded onto +0; NaN below every number) in the high word and
 // the complement of the expert index in the low word (equal logits: the lower
@@ -255,7 +244,8 @@ __device__ void fill_tail(int total, int block_m, int capacity, int32_t* sorted_
 
 // One CTA of 16 warps: optional routing of all T tokens (logits staged in
 // shared memory when they fit), then the whole permutation of A = T*k <=
-// kChunk assignments.
+// kChunk assignments; for FP8 batches with a small x, also amax(x) and the
+// e4m3 codes of x.
 template <int EPL>
 __global__ void __launch_bounds__(kSmallThreads)
     route_permute_small_kernel(const float* __restrict__ logits, int T, int E, int k, int block_m,
@@ -263,7 +253,7 @@ __global__ void __launch_bounds__(kSmallThreads)
                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                int32_t* tiles, int32_t* num_tiles, int32_t* status, int32_t* ctl,
                                int ctl_ints, const uint4* __restrict__ x, long x_vecs,
-                               uint32_t* amax_out) {
+                               uint32_t* amax_out, uint2* __restrict__ xq_out) {
     constexpr int NW = kSmallThreads / 32;
     __shared__ int hist[NW][kMaxExperts];
     __shared__ float slog[kStageFloats];
@@ -302,9 +292,16 @@ __global__ void __launch_bounds__(kSmallThreads)
     }
     chunk_histogram<NW, kChunk>(sids, A, 0, E, hist, status);
     __syncthreads();
-    if (amax_out && threadIdx.x == 0) {
+    if (amax_out) {
         for (int i = 0; i < NW; ++i) xm = fmaxf(xm, wmax[i]);
-        *amax_out = __float_as_uint(xm);
+        if (threadIdx.x == 0) *amax_out = __float_as_uint(xm);
+        // and the e4m3 codes of x (token order), which the gate/up GEMM gathers
+        if (xq_out) {
+            const float sx = fp8_scale_from_amax(__float_as_uint(xm));
+            const float inv = 1.0f / sx;
+            for (long i = threadIdx.x; i < x_vecs; i += kSmallThreads)
+                xq_out[i] = quant8(x[i], inv, sx);
+        }
     }
     const int e = threadIdx.x;
     int c = 0;
@@ -431,13 +428,14 @@ cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k,
                                        int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                        int32_t* tiles, int32_t* num_tiles, int32_t* status,
                                        cudaStream_t s, int32_t* ctl, int ctl_ints, const void* x,
-                                       long x_elems, uint32_t* amax_out) {
+                                       long x_elems, uint32_t* amax_out, void* xq_out) {
     const uint4* xv = static_cast<const uint4*>(x);
+    uint2* xq = static_cast<uint2*>(xq_out);
     const long nv = x_elems / 8;
 #define MOE_SMALL(EPL)                                                                            \
     return launch_pdl(route_permute_small_kernel<EPL>, dim3(1), dim3(kSmallThreads), 0, s, logits, \
                       T, E, k, block_m, capacity, ids, w, counts, offsets, sorted_ids, inv_perm,  \
-                      tiles, num_tiles, status, ctl, ctl_ints, xv, nv, amax_out)
+                      tiles, num_tiles, status, ctl, ctl_ints, xv, nv, amax_out, xq)
     switch (epl_for(E)) {
         case 1: MOE_SMALL(1);
         case 2: MOE_SMALL(2);

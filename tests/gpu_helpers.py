@@ -10,8 +10,8 @@ W_RTOL = 1e-6                      # routing weights
 
 
 def lib():
-    from mixture_experts_expert_route_b200 import build
-    build.build()
+    from mixture_experts_expert_route_b200 import _lib, build
+    build.build(debug=_lib.DEBUG_CHECKS)
     import mixture_experts_expert_route_b200 as moe
     return moe
 

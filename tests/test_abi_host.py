@@ -15,8 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def L():
-    from mixture_experts_expert_route_b200 import build
-    build.build()
+    from mixture_experts_expert_route_b200 import _lib, build
+    build.build(debug=_lib.DEBUG_CHECKS)
     import mixture_experts_expert_route_b200 as moe
     return moe
 
@@ -97,7 +97,7 @@ def test_argument_errors_return_synchronously(L):
 def _fwd(L, **kw):
     base = dict(dtype=0, T=4, k=2, E=8, H=256, I=512, block_m=16, x=0x1000, logits=0x1000,
                 packed=0x1000, scales=None, out=0x1000, ids=None, w=None, status=None,
-                max_ctas=0, events=None, n_events=0)
+                max_ctas=0, events=None, n_events=0, combine=0)
     base.update(kw)
     a = L._lib.ForwardArgs(*[base[f] for f, _ in L._lib.ForwardArgs._fields_])
     return a
@@ -120,6 +120,8 @@ def test_forward_argument_errors(L):
     assert call(_fwd(L, logits=None)) == INVALID
     assert call(_fwd(L, max_ctas=-1)) == INVALID
     assert call(_fwd(L, events=0x1000, n_events=3)) == INVALID
+    assert call(_fwd(L, combine=3)) == INVALID                # unknown combine mode
+    assert call(_fwd(L, combine=-1)) == INVALID
     assert call(_fwd(L), 64) == WS                            # workspace too small
     assert call(_fwd(L, T=0, x=None, logits=None)) == 0       # T = 0 no-op
     assert lib.moe_forward(None, ws, big, None) == INVALID

@@ -72,9 +72,11 @@ def test_bench_mirrors_library_dispatch_constants():
     assert bench.SMALL_T == const("kSmallT")
     assert bench.CHUNK == const("kChunk")
     assert bench.SMALL_AMAX == const("kSmallAmaxElems")
-    # decode T=1 (small path, bf16): route+permute, gather, gate/up, down, combine
-    assert bench.kernels_per_forward(1, 2, False, 4096) == 5
-    # FP8 T=1, x of 5.6 KB: amax folded into the route kernel, plus h quantisation
-    assert bench.kernels_per_forward(1, 4, True, 2880) == 6
-    # FP8 T=2048: route, 3 permutation kernels, amax, gather, 2 GEMMs, quant, combine
+    # decode T=1 (small path, bf16): route+permute, gate/up, down, combine
+    assert bench.kernels_per_forward(1, 2, False, 4096) == 4
+    # FP8 T=1, x of 5.6 KB: amax and x codes in the route kernel, plus h quantisation
+    assert bench.kernels_per_forward(1, 4, True, 2880) == 5
+    # FP8 T=2048: route, 3 permutation kernels, amax, x codes, 2 GEMMs, quant, finalize
     assert bench.kernels_per_forward(2048, 4, True, 2880) == 10
+    # prefill bf16 T=4096: route, 3 permutation kernels, 2 GEMMs, finalize
+    assert bench.kernels_per_forward(4096, 8, False, 2048) == 7

@@ -114,7 +114,7 @@ def test_pack_weights_fp8_codes(moe):
     assert torch.equal(to_host(packed), ref)
 
 
-def run_forward(moe, dtype, L, block_m=0, max_ctas=0, ws=None):
+def run_forward(moe, dtype, L, block_m=0, max_ctas=0, ws=None, combine=0):
     Wg, Wu, Wd = (W.to(DEV) for W in L.weights_bf16())
     packed, scales = moe.pack_weights(dtype, Wg, Wu, Wd)
     x = L.x.to(DEV)
@@ -123,7 +123,7 @@ def run_forward(moe, dtype, L, block_m=0, max_ctas=0, ws=None):
     w = torch.empty((L.T, L.k), dtype=torch.float32, device=DEV)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
     out = moe.forward(dtype, x, logits, packed, scales, L.E, L.I, L.k, ids=ids, w=w, status=st,
-                      block_m=block_m, max_ctas=max_ctas, ws=ws)
+                      block_m=block_m, max_ctas=max_ctas, ws=ws, combine=combine)
     assert moe.check_status(st) == 0
     return out, ids, w
 
@@ -137,42 +137,52 @@ LAYER_CASES = [
     ("tiny", 5, 16, 16, 128, 128),       # k = E: every expert
     ("tiny", 700, 2, 1, 192, 128),       # two token tiles per expert (256 + ragged)
     ("tiny", 9, 1, 1, 256, 256),         # E = 1: dense SwiGLU
+    ("tiny", 40, 2, 2, 256, 256),        # pair tiles, token cap 2*mean = 80 (not a multiple of 32)
+    ("tiny", 56, 2, 2, 192, 128),        # pair tiles, 2*mean = 112
 ]
 
 
+# the two forms of the combine: y_perm rows summed in j order, and the
+# down GEMM's epilogue reducing into an fp32 token-order accumulator
+COMBINES = [1, 2]
+
+
+@pytest.mark.parametrize("combine", COMBINES)
 @pytest.mark.parametrize("dtype", [0, 1])
 @pytest.mark.parametrize("case", LAYER_CASES)
-def test_forward_small(moe, dtype, case):
+def test_forward_small(moe, dtype, case, combine):
     name, T, E, k, H, I = case
     L = make_layer(name, T=T, E=E, k=k, H=H, I=I, seed=T + E)
-    out, ids, w = run_forward(moe, dtype, L)
+    out, ids, w = run_forward(moe, dtype, L, combine=combine)
     ids_o, w_o = check_routing(ids, w, L.logits)
     g, u, d = L.weights_bf16()
     ref = oracle_layer(dtype, L.x, ids_o, w_o, g, u, d)
     assert_close(out, ref, dtype, f"{case} dtype={dtype}")
 
 
+@pytest.mark.parametrize("combine", COMBINES)
 @pytest.mark.parametrize("max_ctas", [1, 3, 7, 13, 64])
 @pytest.mark.parametrize("dtype", [0, 1])
-def test_forward_stream_k_splits(moe, dtype, max_ctas):
+def test_forward_stream_k_splits(moe, dtype, max_ctas, combine):
     """Capped grids cut units mid-K: the fixed-order partial reduction must
     give the same result as the oracle and as the uncapped grid."""
     L = make_layer("tiny", T=45, E=6, k=2, H=384, I=256, seed=5)
-    out, ids, w = run_forward(moe, dtype, L, max_ctas=max_ctas)
+    out, ids, w = run_forward(moe, dtype, L, max_ctas=max_ctas, combine=combine)
     ids_o, w_o = check_routing(ids, w, L.logits)
     g, u, d = L.weights_bf16()
     ref = oracle_layer(dtype, L.x, ids_o, w_o, g, u, d)
     assert_close(out, ref, dtype, f"max_ctas={max_ctas}")
 
 
+@pytest.mark.parametrize("combine", COMBINES)
 @pytest.mark.parametrize("max_ctas", [2, 7, 14, 0])
 @pytest.mark.parametrize("dtype", [0, 1])
-def test_forward_cta_pair_splits(moe, dtype, max_ctas):
+def test_forward_cta_pair_splits(moe, dtype, max_ctas, combine):
     """Large token tiles run on CTA pairs (M = 256 per MMA): odd weight-tile
     counts (5 gate/up, 3 down tiles), ragged token tiles and capped grids that
     split pair units stream-K style."""
     L = make_layer("tiny", T=600, E=4, k=2, H=384, I=320, seed=6)
-    out, ids, w = run_forward(moe, dtype, L, max_ctas=max_ctas)
+    out, ids, w = run_forward(moe, dtype, L, max_ctas=max_ctas, combine=combine)
     ids_o, w_o = check_routing(ids, w, L.logits)
     g, u, d = L.weights_bf16()
     ref = oracle_layer(dtype, L.x, ids_o, w_o, g, u, d)
@@ -188,19 +198,41 @@ def test_forward_block_m_variants(moe, block_m):
     assert_close(out, oracle.moe_layer(L.x, ids_o, w_o, g, u, d), 0, f"block_m={block_m}")
 
 
-def test_forward_deterministic(moe):
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_forward_deterministic(moe, dtype):
+    """The deterministic combine (and the fixed-order stream-K reduction) give
+    bit-identical outputs run after run."""
     L = make_layer("tiny", T=200, E=8, k=2, H=256, I=256, seed=2)
-    outs = [run_forward(moe, 0, L, max_ctas=11)[0] for _ in range(10)]
+    outs = [run_forward(moe, dtype, L, max_ctas=11, combine=1)[0] for _ in range(10)]
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
 
 
-def test_fp8_zero_input(moe):
+def test_combine_auto_picks_by_size(moe):
+    """Auto is the deterministic form for small batches (T*k < 4096) and the
+    fused reduction for large ones; each matches its explicit mode."""
+    for T, k, expect in ((100, 2, 1), (1100, 4, 2)):
+        L = make_layer("tiny", T=T, E=8, k=k, H=256, I=256, seed=T)
+        auto = run_forward(moe, 0, L, combine=0)[0]
+        ref = run_forward(moe, 0, L, combine=expect)[0]
+        ids_o, w_o = oracle.route_topk(L.logits, k)
+        g, u, d = L.weights_bf16()
+        assert_close(auto, oracle.moe_layer(L.x, ids_o, w_o, g, u, d), 0, f"auto T={T}")
+        if expect == 1:
+            assert torch.equal(auto, ref)
+        else:
+            # fused sums follow the schedule's order: equal up to rounding
+            diff = (auto.float() - ref.float()).abs().max().item()
+            assert diff <= 1e-2 * ref.float().abs().max().item()
+
+
+@pytest.mark.parametrize("combine", COMBINES)
+def test_fp8_zero_input(moe, combine):
     """x = 0: amax = 0 gives s_x = 1 (and then h = 0, s_h = 1); the output is
     exactly zero, as the oracle's."""
     L = make_layer("tiny", T=24, E=8, k=2, H=256, I=256, seed=3)
     L.x = torch.zeros_like(L.x)
-    out, ids, w = run_forward(moe, 1, L)
+    out, ids, w = run_forward(moe, 1, L, combine=combine)
     ids_o, w_o = check_routing(ids, w, L.logits)
     g, u, d = L.weights_bf16()
     ref, _, (sx, sh) = oracle.moe_layer_fp8(L.x, ids_o, w_o, g, u, d)
@@ -227,8 +259,9 @@ def test_fp8_amax_element_saturates(moe, amax):
     assert_close(out, ref, 1, f"planted amax {amax}")
 
 
+@pytest.mark.parametrize("combine", COMBINES)
 @pytest.mark.parametrize("dtype", [0, 1])
-def test_nonfinite_logits(moe, dtype):
+def test_nonfinite_logits(moe, dtype, combine):
     """Tokens with NaN, -inf and +inf logits: routing stays bit-exact (NaN
     ranks last, -inf below every number); a +inf selection makes that token's
     weights NaN (exp(inf - inf)) on both sides, and only that token's output;
@@ -242,7 +275,7 @@ def test_nonfinite_logits(moe, dtype):
     lg[8, :6] = float("-inf")            # two finite logits left: they are chosen
     lg[9, 4] = float("inf")
     L.logits = lg
-    out, ids, w = run_forward(moe, dtype, L)
+    out, ids, w = run_forward(moe, dtype, L, combine=combine)
     ids_o, w_o = check_routing(ids, w, lg)
     bad = ~np.isfinite(w_o).all(axis=1)
     assert bad.tolist() == [t == 9 for t in range(L.T)]
@@ -279,6 +312,6 @@ def test_components_compose_to_forward(moe):
     y, _ = moe.grouped_ffn(0, x, w.view(-1), perm, packed, scales, L.E, L.I, L.k, status=st)
     out = moe.combine(y, perm["inv_perm"], L.T, L.k, L.H)
     assert moe.check_status(st) == 0
-    ref = moe.forward(0, x, lg, packed, scales, L.E, L.I, L.k)
+    ref = moe.forward(0, x, lg, packed, scales, L.E, L.I, L.k, combine=moe.COMBINE_DETERMINISTIC)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
