@@ -151,9 +151,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Fire-and-forget fp32 add in global memory (performed at L2).
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+// Fire-and-forget add of 4 consecutive fp32 values (16-byte aligned) in
+// global memory, performed at L2 as one operation.
+__device__ __forceinline__ void red_add_v4(float* addr, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
 // ------------------------------------------------------------------ PDL

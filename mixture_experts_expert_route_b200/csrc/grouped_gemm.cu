@@ -31,9 +31,10 @@
 //
 // Roles (512 threads): warp 0 = copy producer (weights; the down kernel's
 // activation rows by TMA), warp 1 = MMA issuer (single thread), warp 2 =
-// TMEM allocator, then (gate/up) the gather forwarder, warps 4-11 = epilogue
-// (two warps per 32-lane TMEM quarter, alternating 16-column chunks), warps
-// 12-15 = gather of the gate/up kernel's token rows (cp.async).
+// TMEM allocator, then (gate/up pairs, rank-1 CTA) the gather forwarder,
+// warps 4-11 = epilogue (two warps per 32-lane TMEM quarter, alternating
+// 16-column chunks), warps 12-15 = gather of the gate/up kernel's token rows
+// (cp.async).
 // Shared-memory ring of stages of KPS k-blocks (A KPS*16 KB + B KPS*rows*128 B,
 // 128-byte swizzle): 2 stages of 4 k-blocks on one CTA (token tiles of at most
 // 64 rows), 3 stages of 2 k-blocks per CTA of a pair (larger tiles).  Two TMEM
@@ -49,9 +50,9 @@
 // shared-memory image of one stage, so a stage's A operand (one to four
 // consecutive k-blocks) is one contiguous copy.  The gate/up kernel's token
 // rows (B) are gathered with 16-byte cp.async copies placed in the same
-// swizzled layout (zero-filled for pads); a forwarder thread waits for them,
-// makes them visible to the tensor core's (async) proxy and arrives on the
-// MMA's barrier.  The down kernel's rows (h, already in permuted order) come
+// swizzled layout (zero-filled for pads); the MMA issuer waits for them,
+// makes them visible to the tensor core's (async) proxy and issues (the
+// rank-1 CTA of a pair forwards its rows' completion the same way).  The down kernel's rows (h, already in permuted order) come
 // through TMA tensor maps with 128-, 64- and 16-row boxes.  Launched with
 // programmatic dependent launch: the producer fetches the first weight tiles
 // before waiting for the previous kernel, whose outputs it loads after.
@@ -75,15 +76,15 @@ constexpr int kEpiThreads = 256;
 constexpr int kGatherWarp0 = 12;      // warps 12..15 gather the gate/up token rows
 constexpr int kGatherLanes = 128;
 constexpr int kGatherRowsPerPass = kGatherLanes / 8;   // 8 lanes per 128-byte row
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 8;
 constexpr int kMinKbPerCta = 4;
-constexpr int kStagingBytes = 8 * 1024;
+constexpr int kStagingBytes = 16 * 1024;   // 2 KB per epilogue warp
 constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
 constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
 struct GemmArgs {
     int E, Mw, K, KB, MT, MTu, Mvalid;   // MTu: weight tiles per unit step (MT, or pairs)
-    int nmax, tmem_cols;
+    int nmax, tmem_cols, stages;
     const uint8_t* a_tiles;
     int ldo;
     void* out;
@@ -138,8 +139,8 @@ struct Seg {
 
 constexpr int kDynSmemMax = kSmemCap - static_cast<int>(sizeof(Ctl)) - 1024;
 
-template <bool PAIR>
-__host__ __device__ constexpr int stages_for() { return PAIR ? 3 : 2; }
+// k-blocks per pipeline stage; the number of stages is as many as fit in
+// shared memory (at most kMaxStages)
 template <bool PAIR>
 __host__ __device__ constexpr int kps_for() { return PAIR ? 2 : 4; }
 
@@ -302,17 +303,32 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
         }
         __syncwarp();
     } else {
-        // lane = output column: each warp-wide add covers 32 consecutive
-        // floats (one 128-byte line) of one token's accumulator row
-        const int hcol = m_own * kBM + 32 * q + lane;
-        float* acc = static_cast<float*>(g.out);
+        // w * y staged as [16 tokens][32 columns] fp32, then added into the
+        // accumulator 16 bytes at a time: each lane adds 4 consecutive
+        // columns of one token's row (a warp-wide add covers four 128-byte
+        // row segments), a quarter of the L2 operations of scalar adds
+        float* st = reinterpret_cast<float*>(staging + ew * 2048);
+        int tok_of_row = -1;   // lane r < 16 holds the token of chunk row r
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float wi = __shfl_sync(kFull, wreg[i & 7], (c0 + i) >> 3);
             const int ti = __shfl_sync(kFull, treg[i & 7], (c0 + i) >> 3);
-            if (ti >= 0 && hcol < g.Mvalid)
-                red_add_f32(acc + static_cast<long>(ti) * g.ldo + hcol, v[i] * wi);
+            if (lane == i) tok_of_row = ti;
+            st[i * 32 + lane] = v[i] * wi;
         }
+        __syncwarp();
+        const int hcol0 = m_own * kBM + 32 * q;
+        float* acc = static_cast<float*>(g.out);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int piece = lane + 32 * t;
+            const int row = piece >> 3, seg = piece & 7;
+            const int ti = __shfl_sync(kFull, tok_of_row, row);
+            if (ti >= 0 && hcol0 < g.Mvalid)
+                red_add_v4(acc + static_cast<long>(ti) * g.ldo + hcol0 + 4 * seg,
+                           *reinterpret_cast<const float4*>(st + row * 32 + 4 * seg));
+        }
+        __syncwarp();
     }
 }
 
@@ -323,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
     constexpr bool GATHER = EPI == 0;
-    constexpr int S = stages_for<PAIR>();
+    const int S = g.stages;
     // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
     constexpr int KPS = kps_for<PAIR>();
     extern __shared__ uint8_t dsmem_raw[];
@@ -382,9 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 31) ctl.scan_tmp[warp] = inc;
         if (threadIdx.x == 0) {
             for (int i = 0; i < S; ++i) {
-                // gate/up: the producer's weight copies plus one forwarded
-                // arrival per CTA for the gathered rows
-                mbar_init(&ctl.full[i], GATHER ? 1 + (PAIR ? 2 : 1) : 1);
+                // gate/up pair: the producer's weight copies plus the peer
+                // CTA's forwarded arrival for its gathered rows (the MMA
+                // thread waits for its own CTA's rows on gfull)
+                mbar_init(&ctl.full[i], GATHER && PAIR ? 2 : 1);
                 mbar_init(&ctl.empty[i], 1);
                 mbar_init(&ctl.gfull[i], kGatherLanes);
             }
@@ -592,31 +609,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t cs = static_cast<uint32_t>((c ^ (r0 & 7)) << 4);
             constexpr int kMaxRowIters = 128 / kGatherRowsPerPass;   // 8
             const uint32_t smB_u32 = smem_u32(smB);
-            pdl_wait();   // sorted_ids and the source rows come from earlier kernels
-            int st = 0;
-            uint32_t par = 1;
-            Cursor cur = cursor();
-            int u, kb0, kb1;
-            bool ok = true;
-            while (ok && active && cur.next(u, kb0, kb1)) {
-                const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
+            // token (row of the source) of each of this lane's rows of a
+            // unit, -1 for pads and rows past the tile
+            auto load_tokens = [&](const Seg& sg, int (&tok)[kMaxRowIters]) {
                 const int rows = PAIR ? sg.Nm / 2 : sg.N;
                 const int first = rank * rows;     // this CTA's first row of the tile
-                long long src_off[kMaxRowIters];
 #pragma unroll
                 for (int i = 0; i < kMaxRowIters; ++i) {
                     const int r = r0 + kGatherRowsPerPass * i;
                     int sid = -1;
-                    if (r < rows && first + r < sg.N) sid = __ldg(g.sorted_ids + sg.b_row + first + r);
+                    if (r < rows && first + r < sg.N)
+                        sid = __ldg(g.sorted_ids + sg.b_row + first + r);
                     if constexpr (kDebugChecks) {
                         if (sid < -1 || sid >= g.A) {
                             report(g.status, MOE_ERR_DEVICE);
                             sid = -1;
                         }
                     }
-                    src_off[i] = sid >= 0 ? static_cast<long long>(sid / g.ktop) * g.src_row_bytes
-                                          : -1;
+                    tok[i] = sid >= 0 ? sid / g.ktop : -1;
                 }
+            };
+            pdl_wait();   // sorted_ids and the source rows come from earlier kernels
+            int st = 0;
+            uint32_t par = 1;
+            Cursor cur = cursor();
+            int u, kb0, kb1;
+            bool ok = true;
+            bool have = active && cur.next(u, kb0, kb1);
+            Seg sg{};
+            int tok[kMaxRowIters];
+            if (have) {
+                sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
+                load_tokens(sg, tok);
+            }
+            while (ok && have) {
+                // the next unit's token rows are fetched while this unit's
+                // stages are issued, so no unit starts with a dependent load
+                int nu, nkb0, nkb1;
+                const bool have_next = cur.next(nu, nkb0, nkb1);
+                Seg nsg{};
+                int ntok[kMaxRowIters];
+#pragma unroll
+                for (int i = 0; i < kMaxRowIters; ++i) ntok[i] = -1;
+                bool fetched = false;
+                const int rows = PAIR ? sg.Nm / 2 : sg.N;
                 for (int kb = sg.kb0; kb < sg.kb1; kb += KPS) {
                     const int nk = min(KPS, sg.kb1 - kb);
                     if (!mbar_wait(&ctl.empty[st], par, &ctl.abort)) {
@@ -632,9 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < kMaxRowIters; ++i) {
                             const int r = r0 + kGatherRowsPerPass * i;
                             if (r < rows) {
-                                const bool v = in_row && src_off[i] >= 0;
-                                const uint8_t* src = v ? g.gather_src + src_off[i] + kofs
-                                                       : g.gather_src;
+                                const bool v = in_row && tok[i] >= 0;
+                                const uint8_t* src =
+                                    v ? g.gather_src + static_cast<long long>(tok[i]) * g.src_row_bytes + kofs
+                                      : g.gather_src;
                                 cp_async16(dst0 + r * kRowBytes, src, v ? 16u : 0u);
                             }
                         }
@@ -644,6 +681,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         st = 0;
                         par ^= 1u;
                     }
+                    if (!fetched && have_next) {
+                        nsg = make_seg<PAIR>(ctl, g, nu, nkb0, nkb1);
+                        load_tokens(nsg, ntok);
+                        fetched = true;
+                    }
+                }
+                have = have_next;
+                if (have) {
+                    if (!fetched) {
+                        nsg = make_seg<PAIR>(ctl, g, nu, nkb0, nkb1);
+                        load_tokens(nsg, ntok);
+                    }
+                    sg = nsg;
+#pragma unroll
+                    for (int i = 0; i < kMaxRowIters; ++i) tok[i] = ntok[i];
                 }
             }
             // no copy may still target shared memory when the CTA moves on
@@ -651,12 +703,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kFwdWarp) {
         // ------------------------------------------------ gather forwarder
-        // Waits until a stage's gathered rows have landed in this CTA's
-        // shared memory, makes them visible to the async proxy (the tensor
-        // core reads operands through it) and arrives on the MMA issuer's
-        // barrier (the rank-0 CTA's, for a pair).
-        if constexpr (GATHER) {
-            if (lane == 0) {
+        // In the rank-1 CTA of a pair: waits until a stage's gathered rows
+        // have landed in this CTA's shared memory, makes them visible to the
+        // async proxy (the tensor core reads operands through it) and
+        // arrives on the rank-0 CTA's barrier, where the MMA issuer waits.
+        // (The MMA issuer handles its own CTA's rows the same way itself.)
+        if constexpr (GATHER && PAIR) {
+            if (lane == 0 && rank == 1) {
                 int st = 0;
                 uint32_t ph = 0;
                 Cursor cur = cursor();
@@ -670,8 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         fence_proxy_async_smem();
-                        if constexpr (PAIR) mbar_arrive_cluster(leader_addr(&ctl.full[st]));
-                        else mbar_arrive_cluster(smem_u32(&ctl.full[st]));
+                        mbar_arrive_cluster(leader_addr(&ctl.full[st]));
                         if (++st == S) {
                             st = 0;
                             ph ^= 1u;
@@ -712,9 +764,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = make_idesc<FP8>(PAIR ? 2 * kBM : kBM, s.Nm);
                 for (int kb = s.kb0; kb < s.kb1; kb += KPS, ++it) {
                     const int nk = s.kb1 - kb;
-                    // gathered rows arrive through a release at cluster scope
-                    const bool got = GATHER ? mbar_wait_cluster(&ctl.full[st], ph, &ctl.abort)
-                                            : mbar_wait(&ctl.full[st], ph, &ctl.abort);
+                    bool got = true;
+                    if constexpr (GATHER) {
+                        // this CTA's gathered rows: wait for their copies,
+                        // then make them visible to the tensor core's proxy
+                        got = mbar_wait(&ctl.gfull[st], ph, &ctl.abort);
+                        if (got) fence_proxy_async_smem();
+                    }
+                    // weights (and, for a pair, the peer's forwarded rows,
+                    // released at cluster scope)
+                    if (got)
+                        got = GATHER && PAIR ? mbar_wait_cluster(&ctl.full[st], ph, &ctl.abort)
+                                             : mbar_wait(&ctl.full[st], ph, &ctl.abort);
                     if (!got) {
                         raise_abort(ctl, g.status);
                         ok = false;
@@ -1084,10 +1145,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     // fewer, larger copies sustain more bandwidth than many 16 KB stages, for
     // both regimes.
     const int kps = pair ? kps_for<true>() : kps_for<false>();
-    const int stages = pair ? stages_for<true>() : stages_for<false>();
     const int stage_bytes = kps * (kATileBytes + (pair ? p.nmax / 2 : p.nmax) * kRowBytes);
+    int stages = (kDynSmemMax - 1024 - kStagingBytes) / stage_bytes;
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return cudaErrorInvalidValue;
     const int smem = 1024 + stages * stage_bytes + kStagingBytes;
-    if (smem > kDynSmemMax) return cudaErrorInvalidValue;
+    g.stages = stages;
     g.tmem_cols = pow2_at_least(2 * p.nmax);
     g.ldo = p.ldo;
     g.out = p.out;
