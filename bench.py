@@ -4,8 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all]
                     [--impl native|reference]
 
-A step is one pass of the whole layer (route -> permute -> gate/up GEMM with
-the gather of x fused in -> [FP8 h quant] -> down GEMM -> combine) over one
+A step is one pass of the whole layer (route -> permute -> [gather] -> gate/up
+GEMM -> [FP8 h quant] -> down GEMM -> combine) over one
 batch of every token count of a workload, e.g. T = 1, 4, 16, 64 for the
 decode workload (H=4096, I=14336, E=8, top-2, bf16).  Inputs are seeded
 synthetic tensors; the expert weights are larger than the 126 MB L2 and four
@@ -88,7 +88,16 @@ def describe(name):
             f"T={','.join(str(t) for t in c['T'])}")
 
 
-def kernels_per_forward(T, k, fp8, H):
+def gemm_token_cap(T, k, E):
+    """The GEMMs' token-tile cap: twice the mean tokens per expert in steps of
+    16 (16..256), rounded to 32 above 64 (CTA-pair tiles)."""
+    n = max(16, ((2 * T * k + E - 1) // E + 15) // 16 * 16)
+    if n > 64:
+        n = (n + 31) // 32 * 32
+    return min(n, 256)
+
+
+def kernels_per_forward(T, k, E, fp8, H):
     """Kernels one moe_forward launches."""
     A = T * k
     small = T <= SMALL_T and A <= CHUNK
@@ -98,7 +107,8 @@ def kernels_per_forward(T, k, fp8, H):
         n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
     # FP8: amax(x) and the codes of x (in the route kernel for small batches)
     n += 2 if fp8 and not (small and T * H <= SMALL_AMAX) else 0
-    n += 1                                      # gate/up GEMM (gathers x itself)
+    n += 1 if gemm_token_cap(T, k, E) > 64 else 0   # gather (pair tiles; else in the GEMM)
+    n += 1                                      # gate/up GEMM
     n += 1 if fp8 else 0                        # h quantisation
     n += 2                                      # down GEMM + combine (or finalize)
     return n
@@ -629,7 +639,7 @@ class Bench:
                           "double-buffered"}
 
     def launches(self):
-        return self.args.steps * sum(kernels_per_forward(T, self.k, self.fp8, self.H)
+        return self.args.steps * sum(kernels_per_forward(T, self.k, self.E, self.fp8, self.H)
                                      for T in self.Ts)
 
 

@@ -167,10 +167,12 @@ MOE_API moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const 
  * jobban kihasználja a Hopper GPU-kat", re-derived for tcgen05), with the
  * gather of the token rows, the SiLU*up and the routing-weight epilogues
  * fused in:
- *   X_p       = x[sorted_ids[p] / k]      gathered by the gate/up GEMM's
- *                                         operand loads, never stored (zero for
- *                                         pads; FP8: the e4m3 codes of x with
- *                                         s_x = amax(x)/448, made in token order)
+ *   X_p       = x[sorted_ids[p] / k]      zero for pads; FP8: the e4m3 codes
+ *                                         of x with s_x = amax(x)/448, made in
+ *                                         token order.  Tiles of up to 64 tokens
+ *                                         gather X_p in the gate/up GEMM's
+ *                                         operand loads; larger tiles read rows
+ *                                         a gather kernel lays out first
  *   h[p]      = SiLU(X_p W_g[e]) * (X_p W_u[e])   (bf16; FP8: then quantised
  *                                                  with s_h)
  *   y_perm[p] = w[sorted_ids[p]] * (h[p] W_d[e])   (bf16; 0 for pads)
@@ -225,17 +227,20 @@ MOE_API moe_status moe_combine(const void* y_perm, const int32_t* inv_perm, int 
  *   status   optional device status word (NULL: the first int32 of ws)
  *   block_m  0 selects 16
  *   events / n_events  optional: if non-NULL, events[i] is recorded on the
- *            stream after stage i (0 entry, 1 route+permute, 2 FP8 x
- *            quantisation (empty for bf16 and small FP8 batches, where the
- *            route kernel does it), 3 gate/up GEMM, 4 h quant (FP8), 5 down
- *            GEMM, 6 combine or finalize); used to time the stages.  n_events
- *            must be 7 when events is non-NULL.
+ *            stream after stage i (0 entry, 1 route+permute, 2 a3: the FP8
+ *            quantisation of x and, for large token tiles, the gather of the
+ *            token rows (empty when the gate/up GEMM gathers them itself and
+ *            the route kernel quantises x), 3 gate/up GEMM, 4 h quant (FP8),
+ *            5 down GEMM, 6 combine or finalize); used to time the stages.
+ *            n_events must be 7 when events is non-NULL.
  *   combine  a moe_combine_mode (0 = auto).
  * Errors: as for the stages above.
  */
 /* How moe_forward forms out[t] = sum_j y(t, j) (a7). */
 typedef enum {
-    MOE_COMBINE_AUTO = 0,          /* fused for T*k >= 4096, deterministic below */
+    MOE_COMBINE_AUTO = 0,          /* the library's choice: currently the
+                                      deterministic form, which measured as fast
+                                      as the fused one on B200 */
     MOE_COMBINE_DETERMINISTIC = 1, /* the down GEMM writes y_perm rows (bf16); a
                                       combine kernel sums each token's k rows in
                                       fp32 in j order: bit-reproducible */

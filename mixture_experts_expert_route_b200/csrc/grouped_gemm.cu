@@ -29,12 +29,11 @@
 // kernel can add w * y into an fp32 accumulator in token order (the combine)
 // instead of writing permuted rows.
 //
-// Roles (512 threads): warp 0 = copy producer (weights; the down kernel's
-// activation rows by TMA), warp 1 = MMA issuer (single thread), warp 2 =
-// TMEM allocator, then (gate/up pairs, rank-1 CTA) the gather forwarder,
-// warps 4-11 = epilogue (two warps per 32-lane TMEM quarter, alternating
-// 16-column chunks), warps 12-15 = gather of the gate/up kernel's token rows
-// (cp.async).
+// Roles (512 threads): warp 0 = copy producer (weights; activation rows by
+// TMA where they are already in permuted order), warp 1 = MMA issuer (single
+// thread), warp 2 = TMEM allocator, warps 4-11 = epilogue (two warps per
+// 32-lane TMEM quarter, alternating 16-column chunks), warps 12-15 = gather of
+// a one-CTA gate/up kernel's token rows (cp.async).
 // Shared-memory ring of stages of KPS k-blocks (A KPS*16 KB + B KPS*rows*128 B,
 // 128-byte swizzle): 2 stages of 4 k-blocks on one CTA (token tiles of at most
 // 64 rows), 3 stages of 2 k-blocks per CTA of a pair (larger tiles).  Two TMEM
@@ -49,11 +48,17 @@
 // Weights (A) are pre-packed as 16 KB tiles that are already the swizzled
 // shared-memory image of one stage, so a stage's A operand (one to four
 // consecutive k-blocks) is one contiguous copy.  The gate/up kernel's token
-// rows (B) are gathered with 16-byte cp.async copies placed in the same
-// swizzled layout (zero-filled for pads); the MMA issuer waits for them,
-// makes them visible to the tensor core's (async) proxy and issues (the
-// rank-1 CTA of a pair forwards its rows' completion the same way).  The down kernel's rows (h, already in permuted order) come
-// through TMA tensor maps with 128-, 64- and 16-row boxes.  Launched with
+// rows (B) of one-CTA tiles (decode-sized, at most 64 tokens) are gathered
+// with 16-byte cp.async copies placed in the same swizzled layout
+// (zero-filled for pads); the MMA issuer waits for them, makes them visible
+// to the tensor core's (async) proxy and issues.  Rows already in permuted
+// order (the down kernel's h; the gate/up rows of CTA-pair tiles, which a
+// gather kernel lays out first) come through TMA tensor maps with 128-, 64-
+// and 16-row boxes.  Measured on B200: pair tiles gathered by cp.async ran
+// the gate/up GEMM 1.3x slower than TMA from pre-gathered rows (prefill
+// T = 4096: 320 vs 240 us), more than the gather kernel costs, while one-CTA
+// tiles gathered in-kernel match the TMA path and save the gather kernel.
+// Launched with
 // programmatic dependent launch: the producer fetches the first weight tiles
 // before waiting for the previous kernel, whose outputs it loads after.
 #include <cstring>
@@ -70,7 +75,7 @@ constexpr int kBM = 128;            // weight rows per tile (UMMA M)
 constexpr int kRowBytes = 128;      // K bytes per stage row (one swizzle atom)
 constexpr int kATileBytes = kBM * kRowBytes;
 constexpr int kThreads = 512;
-constexpr int kFwdWarp = 2;           // TMEM allocator, then the gather forwarder
+constexpr int kFwdWarp = 2;           // TMEM allocator
 constexpr int kEpiWarp0 = 4;          // warps 4..11: two per TMEM lane quarter
 constexpr int kEpiThreads = 256;
 constexpr int kGatherWarp0 = 12;      // warps 12..15 gather the gate/up token rows
@@ -338,7 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB128,
                         const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
-    constexpr bool GATHER = EPI == 0;
+    // gate/up token rows: gathered by the kernel itself for one-CTA tiles;
+    // CTA-pair tiles (large token tiles) read rows a gather kernel laid out
+    // in permuted order, by TMA
+    constexpr bool GATHER = EPI == 0 && !PAIR;
     const int S = g.stages;
     // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
     constexpr int KPS = kps_for<PAIR>();
@@ -398,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 31) ctl.scan_tmp[warp] = inc;
         if (threadIdx.x == 0) {
             for (int i = 0; i < S; ++i) {
-                // gate/up pair: the producer's weight copies plus the peer
-                // CTA's forwarded arrival for its gathered rows (the MMA
-                // thread waits for its own CTA's rows on gfull)
-                mbar_init(&ctl.full[i], GATHER && PAIR ? 2 : 1);
+                // the producer's copies (the gathered rows of a one-CTA
+                // gate/up kernel complete on gfull, which the MMA thread
+                // waits for itself)
+                mbar_init(&ctl.full[i], 1);
                 mbar_init(&ctl.empty[i], 1);
                 mbar_init(&ctl.gfull[i], kGatherLanes);
             }
@@ -701,38 +709,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             // no copy may still target shared memory when the CTA moves on
             cp_async_wait_all();
         }
-    } else if (warp == kFwdWarp) {
-        // ------------------------------------------------ gather forwarder
-        // In the rank-1 CTA of a pair: waits until a stage's gathered rows
-        // have landed in this CTA's shared memory, makes them visible to the
-        // async proxy (the tensor core reads operands through it) and
-        // arrives on the rank-0 CTA's barrier, where the MMA issuer waits.
-        // (The MMA issuer handles its own CTA's rows the same way itself.)
-        if constexpr (GATHER && PAIR) {
-            if (lane == 0 && rank == 1) {
-                int st = 0;
-                uint32_t ph = 0;
-                Cursor cur = cursor();
-                int u, kb0, kb1;
-                bool ok = true;
-                while (ok && active && cur.next(u, kb0, kb1)) {
-                    for (int kb = kb0; kb < kb1; kb += KPS) {
-                        if (!mbar_wait(&ctl.gfull[st], ph, &ctl.abort)) {
-                            raise_abort(ctl, g.status);
-                            ok = false;
-                            break;
-                        }
-                        fence_proxy_async_smem();
-                        mbar_arrive_cluster(leader_addr(&ctl.full[st]));
-                        if (++st == S) {
-                            st = 0;
-                            ph ^= 1u;
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-        }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && active && rank == 0) {
@@ -771,11 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         got = mbar_wait(&ctl.gfull[st], ph, &ctl.abort);
                         if (got) fence_proxy_async_smem();
                     }
-                    // weights (and, for a pair, the peer's forwarded rows,
-                    // released at cluster scope)
-                    if (got)
-                        got = GATHER && PAIR ? mbar_wait_cluster(&ctl.full[st], ph, &ctl.abort)
-                                             : mbar_wait(&ctl.full[st], ph, &ctl.abort);
+                    // weights (and the TMA-loaded activation rows)
+                    if (got) got = mbar_wait(&ctl.full[st], ph, &ctl.abort);
                     if (!got) {
                         raise_abort(ctl, g.status);
                         ok = false;
@@ -1172,7 +1145,8 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.counters = p.counters;
     g.status = p.status;
     g.sched_after_wait = p.sched_after_wait ? 1 : 0;
-    if (p.epi == 0 && (!p.gather_src || !p.sorted_ids || p.ktop < 1)) return cudaErrorInvalidValue;
+    if (p.epi == 0 && !pair && (!p.gather_src || !p.sorted_ids || p.ktop < 1))
+        return cudaErrorInvalidValue;
     if (p.epi != 0 && (!p.sorted_ids || !p.w)) return cudaErrorInvalidValue;
     if (p.acc_zero_floats % 4 != 0) return cudaErrorInvalidValue;
     CUtensorMap ta, tb128, tb64, tb16;
@@ -1180,11 +1154,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     memset(&tb128, 0, sizeof(tb128));
     memset(&tb64, 0, sizeof(tb64));
     memset(&tb16, 0, sizeof(tb16));
-    // the down kernel's activation rows (h, permuted order) come by TMA; the
-    // gate/up kernel gathers its rows and uses no activation maps
-    if (p.epi != 0 && (!make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
-                       !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
-                       !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16)))
+    // activation rows in permuted order come by TMA; a one-CTA gate/up
+    // kernel gathers its rows itself and uses no activation maps
+    const bool gathers = p.epi == 0 && !pair;
+    if (!gathers && (!p.act || !make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
+                     !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
+                     !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16)))
         return cudaErrorInvalidValue;
     if (pair && !make_tile_map(&ta, p.weights, static_cast<long>(p.E) * p.MT * p.KB, kps))
         return cudaErrorInvalidValue;

@@ -85,6 +85,11 @@ cudaError_t launch_amax_bf16(const void* src, long n, uint32_t* amax_bits, cudaS
 // FP8 x in token order: xq = RNE_sat(x * (1 / s_x)), s_x from amax_bits.
 cudaError_t launch_quant_x_fp8(const void* x, long n, const uint32_t* amax_bits, void* xq,
                                cudaStream_t s);
+// dst[p] = src[sorted_ids[p] / k] (rows of row_bytes, a multiple of 16), pads
+// zero: the permuted token rows of CTA-pair GEMM tiles
+cudaError_t launch_gather_rows(const void* src, int row_bytes, const int32_t* sorted_ids,
+                               const int32_t* offsets, int E, int k, int capacity, void* dst,
+                               cudaStream_t s);
 cudaError_t launch_quant_rows_fp8(const void* h, const int32_t* offsets, int E, int cols,
                                   int capacity, const uint32_t* amax_bits, void* h_q,
                                   cudaStream_t s);
@@ -112,8 +117,9 @@ struct GemmProblem {
     int capacity;         // rows of the permuted operands
     const void* weights;  // packed tiles of this matrix (see PackedGeom)
     int MT, KB;           // row tiles and k-blocks per expert
-    const void* act;      // epi 1/2: [capacity, K] rows in permuted order
-    const void* gather_src;  // epi 0: [T, K] rows in token order
+    const void* act;      // [capacity, K] rows in permuted order (all but the
+                          // one-CTA gate/up kernel, which gathers)
+    const void* gather_src;  // epi 0, one-CTA tiles: [T, K] rows in token order
     void* out;            // epi 0/1: [capacity, ldo] bf16; epi 2: [T, ldo] f32
     int ldo;
     const int32_t* counts;
@@ -134,6 +140,9 @@ struct GemmProblem {
     int sched_after_wait;        // counts/offsets are written by the previous kernel
 };
 int gemm_nmax_for(int T, int k, int E);
+// Token tiles above 64 rows run on CTA pairs (whose gate/up rows are gathered
+// by a separate kernel)
+inline bool gemm_uses_pairs(int nmax) { return nmax > 64; }
 size_t gemm_partials_bytes(int nmax);
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 

@@ -61,6 +61,7 @@ struct Carver {
 struct FfnBuffers {
     int32_t* ctl;
     void* xq;         // FP8: e4m3 codes of x, token order [T, H]
+    void* x_perm;     // CTA-pair tiles: permuted token rows [cap, H] (bf16 / e4m3)
     void* h;
     void* h_q;
     float* partials;
@@ -70,6 +71,8 @@ void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int T, int cap, int 
                     int nmax) {
     const bool fp8 = dt == MOE_FP8_E4M3;
     b.xq = fp8 ? c.take<void>(static_cast<size_t>(T) * H) : nullptr;
+    b.x_perm = gemm_uses_pairs(nmax) ? c.take<void>(static_cast<size_t>(cap) * H * (fp8 ? 1 : 2))
+                                     : nullptr;
     b.h = c.take<void>(static_cast<size_t>(cap) * I * 2);
     b.h_q = fp8 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
     b.partials = c.take<float>(gemm_partials_bytes(nmax));
@@ -137,6 +140,16 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
             return MOE_ERR_CUDA;
         counts_from_prev = false;
     }
+    const void* rows_src = fp8 ? b.xq : f.x;
+    if (gemm_uses_pairs(nmax)) {
+        // large token tiles: lay the token rows out in permuted order for
+        // the pair GEMM's TMA loads
+        Range r("moe: gather (a3)");
+        if (launch_gather_rows(rows_src, f.H * (fp8 ? 1 : 2), f.sorted_ids, f.offsets, f.E, f.k,
+                               f.cap, b.x_perm, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        counts_from_prev = false;
+    }
     record(ev, 2, s);
 
     const PackedGeom geo = packed_geom(fp8, f.E, f.H, f.I);
@@ -153,7 +166,8 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     gu.weights = f.packed;
     gu.MT = geo.mt_gu;
     gu.KB = geo.kb_gu;
-    gu.gather_src = fp8 ? b.xq : f.x;
+    gu.gather_src = rows_src;
+    gu.act = b.x_perm;
     gu.out = b.h;
     gu.ldo = f.I;
     gu.counts = f.counts;
@@ -257,15 +271,12 @@ FwdBuffers carve_fwd(Carver& c, moe_dtype dt, int T, int k, int E, int H, int I,
 
 // The combine a forward call uses.  The gather-sum is deterministic (a fixed
 // summation order); the fused reduction skips the y_perm round trip through
-// memory but adds in arrival order.  Auto picks the fused form where y_perm
-// is large.
-constexpr long kFusedMinAssignments = 4096;
-
-Combine pick_combine(int mode, int T, int k) {
-    if (mode == MOE_COMBINE_DETERMINISTIC) return Combine::kGatherSum;
-    if (mode == MOE_COMBINE_FUSED) return Combine::kFused;
-    return static_cast<long>(T) * k >= kFusedMinAssignments ? Combine::kFused
-                                                           : Combine::kGatherSum;
+// memory but adds in arrival order.  Auto takes the gather-sum: measured on
+// B200, the fused form's L2 reductions slowed the down GEMM by about what
+// they saved (prefill T = 4096: down +21 us, combine -25 us; skewed T = 8192:
+// down +158 us, combine -144 us; FP8 T = 2048: +5 / -4 us).
+Combine pick_combine(int mode) {
+    return mode == MOE_COMBINE_FUSED ? Combine::kFused : Combine::kGatherSum;
 }
 
 }  // namespace
@@ -471,7 +482,7 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     // the single-CTA permutation (the only one for A <= 2048) is the kernel
     // right before the gate/up GEMM, unless FP8 kernels come between
     f.counts_from_prev = permute_chunks(A) <= 1;
-    f.combine = pick_combine(a->combine, a->T, a->k);
+    f.combine = pick_combine(a->combine);
     st = run_ffn(f, b.ffn, ev, s);
     if (st != MOE_OK) return st;
     {

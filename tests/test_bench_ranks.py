@@ -72,11 +72,16 @@ def test_bench_mirrors_library_dispatch_constants():
     assert bench.SMALL_T == const("kSmallT")
     assert bench.CHUNK == const("kChunk")
     assert bench.SMALL_AMAX == const("kSmallAmaxElems")
-    # decode T=1 (small path, bf16): route+permute, gate/up, down, combine
-    assert bench.kernels_per_forward(1, 2, False, 4096) == 4
+    # decode T=1 (small path, bf16): route+permute, gate/up (gathers), down, combine
+    assert bench.kernels_per_forward(1, 2, 8, False, 4096) == 4
     # FP8 T=1, x of 5.6 KB: amax and x codes in the route kernel, plus h quantisation
-    assert bench.kernels_per_forward(1, 4, True, 2880) == 5
-    # FP8 T=2048: route, 3 permutation kernels, amax, x codes, 2 GEMMs, quant, finalize
-    assert bench.kernels_per_forward(2048, 4, True, 2880) == 10
-    # prefill bf16 T=4096: route, 3 permutation kernels, 2 GEMMs, finalize
-    assert bench.kernels_per_forward(4096, 8, False, 2048) == 7
+    assert bench.kernels_per_forward(1, 4, 32, True, 2880) == 5
+    # FP8 T=2048: route, 3 permutation kernels, amax, x codes, gather, 2 GEMMs,
+    # quant, finalize
+    assert bench.kernels_per_forward(2048, 4, 32, True, 2880) == 11
+    # prefill bf16 T=4096: route, 3 permutation kernels, gather, 2 GEMMs, finalize
+    assert bench.kernels_per_forward(4096, 8, 128, False, 2048) == 8
+    # the token-tile cap (pair tiles above 64): twice the mean per expert
+    assert bench.gemm_token_cap(64, 2, 8) == 32
+    assert bench.gemm_token_cap(40, 2, 2) == 96
+    assert bench.gemm_token_cap(4096, 8, 128) == 256

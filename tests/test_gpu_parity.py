@@ -208,10 +208,10 @@ def test_forward_deterministic(moe, dtype):
         assert torch.equal(o, outs[0])
 
 
-def test_combine_auto_picks_by_size(moe):
-    """Auto is the deterministic form for small batches (T*k < 4096) and the
-    fused reduction for large ones; each matches its explicit mode."""
-    for T, k, expect in ((100, 2, 1), (1100, 4, 2)):
+def test_combine_auto_is_deterministic(moe):
+    """Auto takes the deterministic combine at every size: bit-identical to the
+    explicit mode; the fused reduction matches up to rounding."""
+    for T, k, expect in ((100, 2, 1), (1100, 4, 1), (1100, 4, 2)):
         L = make_layer("tiny", T=T, E=8, k=k, H=256, I=256, seed=T)
         auto = run_forward(moe, 0, L, combine=0)[0]
         ref = run_forward(moe, 0, L, combine=expect)[0]
@@ -221,6 +221,7 @@ def test_combine_auto_picks_by_size(moe):
         if expect == 1:
             assert torch.equal(auto, ref)
         else:
+            assert_close(ref, oracle.moe_layer(L.x, ids_o, w_o, g, u, d), 0, f"fused T={T}")
             # fused sums follow the schedule's order: equal up to rounding
             diff = (auto.float() - ref.float()).abs().max().item()
             assert diff <= 1e-2 * ref.float().abs().max().item()
