@@ -50,6 +50,8 @@ def lib():
                                        P, i32, P]
         L.oracle_moe_layer_fp8.argtypes = [i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, i32,
                                            P, i32, P, P, P]
+        L.oracle_moe_layer_lora.argtypes = [i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, i32,
+                                            i32, i32, P, P, P, P, P, P, P, i32, P, P, i32, P]
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_decode.restype = ctypes.c_float
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
@@ -177,6 +179,34 @@ def moe_layer_fp8(x, ids, w, Wg, Wu, Wd, tokens=None):
     if rc != 0:
         raise ValueError(f"oracle_moe_layer_fp8: {rc}")
     return out, ws, (float(acts[0]), float(acts[1]))
+
+
+def moe_layer_lora(x, ids, w, Wg, Wu, Wd, adapter, lora, scale, tokens=None):
+    """Multi-LoRA layer.  adapter: int [T] (-1 = base model); lora: dict of
+    Ag, Au [n_a,E,H,r], Bg, Bu [n_a,E,r,I], Ad [n_a,E,I,r], Bd [n_a,E,r,H]
+    (one dtype); scale: [n_a].  Returns out [n,H] float64."""
+    xa, xdt, ga, ua, da, gdt, ids, w, T, H, I, E, k, tok, n = _layer_args(x, ids, w, Wg, Wu, Wd,
+                                                                          tokens)
+    mats = [_arr(lora[key]) for key in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")]
+    ldt = mats[0][1]
+    if any(m[1] != ldt for m in mats):
+        raise TypeError("adapter matrices must share a dtype")
+    mats = [m[0] if ldt == BF16 else m[0].astype(np.float32, copy=False) for m in mats]
+    n_a, E2, H2, r = mats[0].shape
+    assert E2 == E and H2 == H
+    assert mats[1].shape == (n_a, E, r, I) and mats[4].shape == (n_a, E, I, r)
+    assert mats[5].shape == (n_a, E, r, H)
+    ad = np.ascontiguousarray(np.asarray(adapter, np.int32))
+    assert ad.shape == (T,)
+    sc = np.ascontiguousarray(np.asarray(scale, np.float64))
+    assert sc.shape == (n_a,)
+    out = np.zeros((n, H), np.float64)
+    rc = lib().oracle_moe_layer_lora(T, H, I, E, k, _p(xa), xdt, _p(ids), _p(w), _p(ga), _p(ua),
+                                     _p(da), gdt, n_a, r, _p(ad), *[_p(m) for m in mats], ldt,
+                                     _p(sc), None if tok is None else _p(tok), n, _p(out))
+    if rc != 0:
+        raise ValueError(f"oracle_moe_layer_lora: {rc}")
+    return out
 
 
 def e4m3_decode(codes) -> np.ndarray:

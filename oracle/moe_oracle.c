@@ -239,6 +239,118 @@ int oracle_moe_layer(int T, int H, int I, int E, int k,
     return bad ? -2 : 0;
 }
 
+/* ------------------------------------------------------------ multi-LoRA
+ * Multi-LoRA serving of MoE models ("Amazon SageMaker AIにおける
+ * Mixture-of-Expertsカーネル最適化の深掘り", § "SageMakerを活用したMoEモデルの
+ * デプロイと性能向上戦略"): several fine-tuned variants of one MoE model
+ * ("adapters") share the GPU.  The pages name the technique only; readings:
+ *  L1  token t carries an adapter index a_t in [0, n_adapters), or -1 for the
+ *      base model alone;
+ *  L2  adapter a holds, for every expert e and each of its three matrices, a
+ *      rank-r pair: W_g[e] + s_a A_g[a,e] B_g[a,e] with A_g [H, r] and
+ *      B_g [r, I]; W_u likewise; W_d[e] + s_a A_d[a,e] B_d[a,e] with
+ *      A_d [I, r] and B_d [r, H] (the usual low-rank adaptation, applied to
+ *      the weights the token actually meets);
+ *  L3  s_a is the adapter's scale (alpha / r in the usual convention), an
+ *      input;
+ *  L4  so g = x W_g + s_a (x A_g) B_g and u likewise, h = SiLU(g) * u,
+ *      y = h W_d + s_a (h A_d) B_d; routing and the weighted combine are
+ *      unchanged.
+ * Layouts: A_g, A_u [n_a][E][H][r], B_g, B_u [n_a][E][r][I], A_d [n_a][E][I][r],
+ * B_d [n_a][E][r][H], all of one dtype (l_dtype).
+ */
+static void lora_shrink(int K, int r, const double* v, const void* A, int adt, size_t base,
+                        double* t) {
+    for (int q = 0; q < r; ++q) t[q] = 0.0;
+    for (int c = 0; c < K; ++c) {
+        double vc = v[c];
+        for (int q = 0; q < r; ++q) t[q] += vc * load(A, adt, base + (size_t)c * r + q);
+    }
+}
+
+int oracle_moe_layer_lora(int T, int H, int I, int E, int k,
+                          const void* x, int x_dtype,
+                          const int32_t* ids, const double* w,
+                          const void* Wg, const void* Wu, const void* Wd, int w_dtype,
+                          int n_adapters, int r, const int32_t* adapter,
+                          const void* Ag, const void* Bg, const void* Au, const void* Bu,
+                          const void* Ad, const void* Bd, int l_dtype, const double* scale,
+                          const int32_t* tokens, int n_tokens, double* out) {
+    if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E || n_adapters < 0 || r < 1)
+        return -1;
+    int n = tokens ? n_tokens : T;
+    int bad = 0;
+    size_t hi = (size_t)H * I;
+#pragma omp parallel
+    {
+        double* g = (double*)malloc(sizeof(double) * (size_t)I);
+        double* u = (double*)malloc(sizeof(double) * (size_t)I);
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        double* xt = (double*)malloc(sizeof(double) * (size_t)H);
+        double* tg = (double*)malloc(sizeof(double) * (size_t)r);
+        double* tu = (double*)malloc(sizeof(double) * (size_t)r);
+        double* td = (double*)malloc(sizeof(double) * (size_t)r);
+        if (!g || !u || !h || !xt || !tg || !tu || !td) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int i = 0; i < n; ++i) {
+                int t = tokens ? tokens[i] : i;
+                double* o = out + (size_t)i * H;
+                for (int c = 0; c < H; ++c) o[c] = 0.0;
+                if (t < 0 || t >= T) continue;
+                int a = adapter ? adapter[t] : -1;
+                if (a >= n_adapters) a = -1;
+                for (int c = 0; c < H; ++c) xt[c] = load(x, x_dtype, (size_t)t * H + c);
+                for (int j = 0; j < k; ++j) {
+                    int e = ids[(size_t)t * k + j];
+                    if (e < 0 || e >= E) continue;
+                    double wgt = w[(size_t)t * k + j];
+                    /* base projections */
+                    for (int m = 0; m < I; ++m) { g[m] = 0.0; u[m] = 0.0; }
+                    for (int c = 0; c < H; ++c) {
+                        size_t b = (size_t)e * hi + (size_t)c * I;
+                        for (int m = 0; m < I; ++m) {
+                            g[m] += xt[c] * load(Wg, w_dtype, b + m);
+                            u[m] += xt[c] * load(Wu, w_dtype, b + m);
+                        }
+                    }
+                    /* the adapter's low-rank deltas (L2, L4) */
+                    size_t ae = 0;
+                    if (a >= 0) {
+                        ae = (size_t)a * E + (size_t)e;
+                        lora_shrink(H, r, xt, Ag, l_dtype, ae * (size_t)H * r, tg);
+                        lora_shrink(H, r, xt, Au, l_dtype, ae * (size_t)H * r, tu);
+                        for (int q = 0; q < r; ++q) {
+                            size_t b = ae * (size_t)r * I + (size_t)q * I;
+                            for (int m = 0; m < I; ++m) {
+                                g[m] += scale[a] * tg[q] * load(Bg, l_dtype, b + m);
+                                u[m] += scale[a] * tu[q] * load(Bu, l_dtype, b + m);
+                            }
+                        }
+                    }
+                    for (int m = 0; m < I; ++m) h[m] = silu(g[m]) * u[m];
+                    for (int m = 0; m < I; ++m) {
+                        size_t b = (size_t)e * hi + (size_t)m * H;
+                        for (int c = 0; c < H; ++c) o[c] += wgt * h[m] * load(Wd, w_dtype, b + c);
+                    }
+                    if (a >= 0) {
+                        lora_shrink(I, r, h, Ad, l_dtype, ae * (size_t)I * r, td);
+                        for (int q = 0; q < r; ++q) {
+                            size_t b = ae * (size_t)r * H + (size_t)q * H;
+                            for (int c = 0; c < H; ++c)
+                                o[c] += wgt * scale[a] * td[q] * load(Bd, l_dtype, b + c);
+                        }
+                    }
+                }
+            }
+        }
+        free(g); free(u); free(h); free(xt); free(tg); free(tu); free(td);
+    }
+    return bad ? -2 : 0;
+}
+
 /* ------------------------------------------------------------ FP8 e4m3
  * FP8 per-tensor quantisation [A] § "FP8 esetén…", [C] (FP8 量子化).
  * e4m3 "fn" encoding: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no

@@ -160,6 +160,51 @@ def make_layer(name: str, T: int | None = None, seed: int = 0, device: str = "cp
                  meta=dict(seed=seed, weight_device=device))
 
 
+@dataclass
+class Lora:
+    """Synthetic adapters for multi-LoRA layers (the pages give no adapter
+    shapes): n_adapters rank-r pairs per expert and matrix, bf16.
+    A_g, A_u [n,E,H,r], B_g, B_u [n,E,r,I], A_d [n,E,I,r], B_d [n,E,r,H];
+    scale [n] float32."""
+    Ag: torch.Tensor
+    Bg: torch.Tensor
+    Au: torch.Tensor
+    Bu: torch.Tensor
+    Ad: torch.Tensor
+    Bd: torch.Tensor
+    scale: torch.Tensor
+
+    def as_dict(self):
+        return dict(Ag=self.Ag, Bg=self.Bg, Au=self.Au, Bu=self.Bu, Ad=self.Ad, Bd=self.Bd)
+
+
+def make_lora(E: int, H: int, I: int, n_adapters: int = 4, rank: int = 16, seed: int = 0,
+              device: str = "cpu") -> Lora:
+    """Adapters drawn by Generator(seed): A ~ N(0, 1/sqrt(fan_in)) (std), B ~
+    N(0, 0.1/sqrt(rank)) so each delta is about a tenth of its base matrix's
+    output; scale_a = 1 + a/4."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    n, r = n_adapters, rank
+    mk = lambda shape, std: _normal(gen, shape, std, "cpu", torch.bfloat16).to(device)
+    Ag = mk((n, E, H, r), 1.0 / math.sqrt(H))
+    Bg = mk((n, E, r, I), 0.1 / math.sqrt(r))
+    Au = mk((n, E, H, r), 1.0 / math.sqrt(H))
+    Bu = mk((n, E, r, I), 0.1 / math.sqrt(r))
+    Ad = mk((n, E, I, r), 1.0 / math.sqrt(I))
+    Bd = mk((n, E, r, H), 0.1 / math.sqrt(r))
+    scale = torch.tensor([1.0 + a / 4.0 for a in range(n)], dtype=torch.float32)
+    return Lora(Ag, Bg, Au, Bu, Ad, Bd, scale)
+
+
+def adapter_ids(T: int, n_adapters: int, seed: int = 0, base_share: float = 0.25) -> torch.Tensor:
+    """Adapter of each token, int32 [T]: -1 (base model only) with probability
+    base_share, else uniform over the adapters."""
+    gen = torch.Generator().manual_seed(seed * 7 + 3)
+    u = torch.rand(T, generator=gen)
+    a = torch.randint(0, max(n_adapters, 1), (T,), generator=gen, dtype=torch.int32)
+    return torch.where(u < base_share, torch.full_like(a, -1), a)
+
+
 def random_ids(T: int, E: int, k: int, seed: int = 0, skew: float = 0.0) -> torch.Tensor:
     """Distinct expert ids per token, [T, k] int32: a seeded routing stand-in for
     tests of the permutation alone.  ``skew`` > 0 biases towards low ids."""
