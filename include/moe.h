@@ -160,6 +160,39 @@ MOE_API moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const 
                             moe_stream_t stream);
 
 /*
+ * Multi-LoRA adapters (bf16 layers).  Several fine-tuned variants of one MoE
+ * model share the GPU, each token naming its adapter ("Amazon SageMaker AIに
+ * おけるMixture-of-Expertsカーネル最適化の深掘り", § "SageMakerを活用した
+ * MoEモデルのデプロイと性能向上戦略": multi-LoRA serving of MoE models).  The
+ * pages give no shapes; this library's definition: adapter a has, for every
+ * expert e, rank-r pairs that add s_a A B to each expert matrix the token
+ * meets:
+ *   g = x W_g + s_a (x A_g) B_g,  u likewise,  h = SiLU(g) * u,
+ *   y = h W_d + s_a (h A_d) B_d
+ * with A_g, A_u [n][E][H][r], B_g, B_u [n][E][r][I], A_d [n][E][I][r],
+ * B_d [n][E][r][H] (device bf16, row-major) and n * r <= 64.
+ * moe_pack_lora lays them out once (moe_packed_lora_size bytes, device,
+ * 16-byte aligned).  The layer computes each shrink (x A, h A, for all
+ * adapters at once, kept only in the token's own adapter's columns and
+ * scaled) as one extra 128-row weight tile per expert, and each expand
+ * (... B) as one or two extra k-blocks of the base GEMMs.
+ * Errors: MOE_ERR_INVALID_ARG for bad sizes or pointers, MOE_ERR_UNSUPPORTED
+ * for n * r > 64 or E > 256.
+ */
+typedef struct {
+    int n_adapters;             /* n >= 1 */
+    int rank;                   /* r >= 1, n * r <= 64 */
+    const int32_t* adapter;     /* device i32 [T]: the token's adapter, -1 = none */
+    const void* packed;         /* device, from moe_pack_lora */
+    const float* scale;         /* device f32 [n]: s_a */
+} moe_lora_args;
+
+MOE_API size_t moe_packed_lora_size(int E, int H, int I, int n_adapters, int rank);
+MOE_API moe_status moe_pack_lora(int E, int H, int I, int n_adapters, int rank, const void* Ag,
+                                 const void* Bg, const void* Au, const void* Bu, const void* Ad,
+                                 const void* Bd, void* packed, moe_stream_t stream);
+
+/*
  * a3-a6. Grouped expert FFN over the permuted assignments: the expert GEMMs
  * A[M,K] x B[K,N] ("Ingénierie de kernels Mixture-of-Experts sur Amazon
  * SageMaker AI"), computed with the expert-weight rows in the tensor core's
@@ -234,6 +267,9 @@ MOE_API moe_status moe_combine(const void* y_perm, const int32_t* inv_perm, int 
  *            5 down GEMM, 6 combine or finalize); used to time the stages.
  *            n_events must be 7 when events is non-NULL.
  *   combine  a moe_combine_mode (0 = auto).
+ *   lora     optional adapters (see moe_lora_args); the workspace from
+ *            moe_forward_workspace_size always has room for their shrink
+ *            outputs.
  * Errors: as for the stages above.
  */
 /* How moe_forward forms out[t] = sum_j y(t, j) (a7). */
@@ -267,6 +303,7 @@ typedef struct {
     moe_event_t* events;
     int n_events;
     int combine;               /* a moe_combine_mode */
+    const moe_lora_args* lora; /* optional multi-LoRA adapters (bf16 only), NULL = none */
 } moe_forward_args;
 
 MOE_API size_t moe_forward_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,

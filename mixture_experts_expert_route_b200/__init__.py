@@ -4,12 +4,12 @@ route top-k -> atomic-free permutation -> tcgen05 grouped SwiGLU GEMMs
 (expert-weight rows in the MMA M slot, tokens in N) -> weighted combine,
 behind the C ABI of include/moe.h.  This package is the thin ctypes binding.
 """
-from ._lib import (BF16, COMBINE_AUTO, COMBINE_DETERMINISTIC, COMBINE_FUSED, FP8_E4M3, MoEError, MoELayer, align_permute, check_status, combine,
+from ._lib import (BF16, COMBINE_AUTO, COMBINE_DETERMINISTIC, COMBINE_FUSED, FP8_E4M3, Lora, MoEError, MoELayer, align_permute, check_status, combine,
                    forward, forward_workspace_size, grouped_ffn, grouped_ffn_workspace_size, lib,
                    pack_weights, permute_capacity, route_topk, selftest_wait_timeout,
                    status_string, version, LIB_PATH)
 
-__all__ = ["BF16", "COMBINE_AUTO", "COMBINE_DETERMINISTIC", "COMBINE_FUSED", "FP8_E4M3", "MoEError", "MoELayer", "align_permute", "check_status", "combine",
+__all__ = ["BF16", "COMBINE_AUTO", "COMBINE_DETERMINISTIC", "COMBINE_FUSED", "FP8_E4M3", "Lora", "MoEError", "MoELayer", "align_permute", "check_status", "combine",
            "forward", "forward_workspace_size", "grouped_ffn", "grouped_ffn_workspace_size", "lib",
            "pack_weights", "permute_capacity", "route_topk", "selftest_wait_timeout",
            "status_string", "version", "LIB_PATH"]

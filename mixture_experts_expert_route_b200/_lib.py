@@ -42,11 +42,17 @@ class FfnArgs(ctypes.Structure):
                 ("y_perm", P), ("status", P), ("max_ctas", I32)]
 
 
+class LoraArgs(ctypes.Structure):
+    _fields_ = [("n_adapters", I32), ("rank", I32), ("adapter", P), ("packed", P),
+                ("scale", P)]
+
+
 class ForwardArgs(ctypes.Structure):
     _fields_ = [("dtype", I32), ("T", I32), ("k", I32), ("E", I32), ("H", I32), ("I", I32),
                 ("block_m", I32), ("x", P), ("logits", P), ("packed", P), ("scales", P),
                 ("out", P), ("ids", P), ("w", P), ("status", P), ("max_ctas", I32),
-                ("events", P), ("n_events", I32), ("combine", I32)]
+                ("events", P), ("n_events", I32), ("combine", I32),
+                ("lora", ctypes.POINTER(LoraArgs))]
 
 
 _SIGS = {
@@ -59,6 +65,8 @@ _SIGS = {
     "moe_align_permute_noalloc": ([P, I32, I32, I32, I32, P, P, P, P, P, P, I32, P], I32),
     "moe_packed_weights_size": ([I32, I32, I32, I32], SZ),
     "moe_pack_weights": ([I32, I32, I32, I32, P, P, P, P, P, P], I32),
+    "moe_packed_lora_size": ([I32, I32, I32, I32, I32], SZ),
+    "moe_pack_lora": ([I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P], I32),
     "moe_grouped_ffn_workspace_size": ([I32, I32, I32, I32, I32, I32, I32], SZ),
     "moe_grouped_ffn": ([ctypes.POINTER(FfnArgs), P, SZ, P], I32),
     "moe_combine": ([P, P, I32, I32, I32, P, P], I32),
@@ -187,6 +195,33 @@ def pack_weights(dtype: int, Wg: torch.Tensor, Wu: torch.Tensor, Wd: torch.Tenso
     return packed, scales
 
 
+class Lora:
+    """Packed multi-LoRA adapters on the device (see moe_pack_lora)."""
+
+    def __init__(self, Ag, Bg, Au, Bu, Ad, Bd, scale, stream=None):
+        n, E, H, r = Ag.shape
+        I = Bg.shape[3]
+        for M in (Ag, Bg, Au, Bu, Ad, Bd):
+            if M.dtype != torch.bfloat16 or not M.is_contiguous() or not M.is_cuda:
+                raise ValueError("adapter matrices must be contiguous bf16 CUDA tensors")
+        self.n_adapters, self.rank, self.E, self.H, self.I = n, r, E, H, I
+        size = lib().moe_packed_lora_size(E, H, I, n, r)
+        if size == 0:
+            raise MoEError(2, "moe_packed_lora_size")
+        self.packed = torch.empty(size, dtype=torch.uint8, device=Ag.device)
+        _check(lib().moe_pack_lora(E, H, I, n, r, _ptr(Ag), _ptr(Bg), _ptr(Au), _ptr(Bu),
+                                   _ptr(Ad), _ptr(Bd), _ptr(self.packed), _stream(stream)),
+               "moe_pack_lora")
+        self.scale = scale.to(device=Ag.device, dtype=torch.float32).contiguous()
+
+    def args(self, adapter):
+        """The C struct for tokens whose adapters are `adapter` (device int32 [T])."""
+        if adapter.dtype != torch.int32 or not adapter.is_cuda:
+            raise ValueError("adapter must be a CUDA int32 tensor")
+        return LoraArgs(self.n_adapters, self.rank, _ptr(adapter), _ptr(self.packed),
+                        _ptr(self.scale))
+
+
 def grouped_ffn_workspace_size(dtype, T, k, E, H, I, block_m) -> int:
     return lib().moe_grouped_ffn_workspace_size(dtype, T, k, E, H, I, block_m)
 
@@ -221,10 +256,12 @@ def forward_workspace_size(dtype, T, k, E, H, I, block_m=0) -> int:
 
 def forward(dtype: int, x, logits, packed, scales, E: int, I: int, k: int, out=None, ids=None,
             w=None, status=None, ws=None, block_m: int = 0, max_ctas: int = 0, events=None,
-            combine: int = COMBINE_AUTO, stream=None):
+            combine: int = COMBINE_AUTO, lora=None, adapter=None, stream=None):
     """The whole layer.  ``events`` (7 torch.cuda.Event, optional) are recorded after
     each stage: entry, route+permute, FP8 x quantisation, gate/up, h quant, down,
-    combine.  ``combine``: COMBINE_AUTO, COMBINE_DETERMINISTIC or COMBINE_FUSED."""
+    combine.  ``combine``: COMBINE_AUTO, COMBINE_DETERMINISTIC or COMBINE_FUSED.
+    ``lora`` (a Lora) with ``adapter`` (CUDA int32 [T], -1 = none) applies
+    multi-LoRA adapters (bf16 layers)."""
     T, H = x.shape
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     n = forward_workspace_size(dtype, T, k, E, H, I, block_m)
@@ -238,10 +275,12 @@ def forward(dtype: int, x, logits, packed, scales, E: int, I: int, k: int, out=N
             if e.cuda_event == 0:  # create lazily-initialised events
                 e.record()
         ev_arr = (ctypes.c_void_p * 7)(*[e.cuda_event for e in events])
+    largs = lora.args(adapter) if lora is not None else None
     a = ForwardArgs(dtype, T, k, E, H, I, block_m, _ptr(x), _ptr(logits), _ptr(packed),
                     _ptr(scales), _ptr(out), _ptr(ids), _ptr(w), _ptr(status), max_ctas,
                     ctypes.cast(ev_arr, ctypes.c_void_p) if ev_arr is not None else None,
-                    7 if ev_arr is not None else 0, combine)
+                    7 if ev_arr is not None else 0, combine,
+                    ctypes.pointer(largs) if largs is not None else None)
     _check(lib().moe_forward(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return out

@@ -253,6 +253,62 @@ __global__ void __launch_bounds__(kThreads)
     for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads) dst[i] = src[i];
 }
 
+// Multi-LoRA adapter tiles (see LoraGeom): one 16 KB tile per CTA, element
+// (row rr, k kk) from the section's definition, bf16, swizzled like the
+// weights.  Layouts: A_g, A_u [n][E][H][r], B_g, B_u [n][E][r][I],
+// A_d [n][E][I][r], B_d [n][E][r][H].  grid = (tiles per expert, 1, E).
+template <int SECTION>
+__global__ void __launch_bounds__(kThreads)
+    pack_lora_kernel(const __nv_bfloat16* __restrict__ Ag, const __nv_bfloat16* __restrict__ Bg,
+                     const __nv_bfloat16* __restrict__ Au, const __nv_bfloat16* __restrict__ Bu,
+                     const __nv_bfloat16* __restrict__ Ad, const __nv_bfloat16* __restrict__ Bd,
+                     int E, int H, int I, int r, int R, int per_expert, uint8_t* __restrict__ out) {
+    __shared__ __align__(16) uint8_t tile[kTileBytes];
+    const int ti = blockIdx.x, e = blockIdx.z;
+    for (int idx = threadIdx.x; idx < kTileRows * 64; idx += kThreads) {
+        const int rr = idx % kTileRows, kk = idx / kTileRows;
+        float v = 0.0f;
+        if constexpr (SECTION == 0) {           // shrink_gu: tile = k-block of H
+            const int kg = ti * 64 + kk, slot = rr & 63;
+            if (kg < H && slot < R) {
+                const int a = slot / r, q = slot % r;
+                const __nv_bfloat16* A = rr < 64 ? Ag : Au;
+                v = __bfloat162float(A[((static_cast<long>(a) * E + e) * H + kg) * r + q]);
+            }
+        } else if constexpr (SECTION == 1) {    // expand_gu: tile = (m, x)
+            const int m = ti >> 1, x = ti & 1;
+            const int Rp = m * kTileRows + rr;
+            const int j = 16 * (Rp / 32) + (Rp & 15);
+            const bool up = (Rp & 31) >= 16;
+            if (Rp < 2 * I && kk < R && up == (x == 1)) {
+                const int a = kk / r, q = kk % r;
+                const __nv_bfloat16* B = up ? Bu : Bg;
+                v = __bfloat162float(B[((static_cast<long>(a) * E + e) * r + q) * I + j]);
+            }
+        } else if constexpr (SECTION == 2) {    // shrink_d: tile = k-block of I
+            const int kg = ti * 64 + kk;
+            if (kg < I && rr < R) {
+                const int a = rr / r, q = rr % r;
+                v = __bfloat162float(Ad[((static_cast<long>(a) * E + e) * I + kg) * r + q]);
+            }
+        } else {                                // expand_d: tile = m
+            const int c = ti * kTileRows + rr;
+            if (c < H && kk < R) {
+                const int a = kk / r, q = kk % r;
+                v = __bfloat162float(Bd[((static_cast<long>(a) * E + e) * r + q) * H + c]);
+            }
+        }
+        const int o = rr * kTileRowBytes + kk * 2;
+        const int sw = o ^ (((o >> 7) & 7) << 4);
+        *reinterpret_cast<__nv_bfloat16*>(tile + sw) = __float2bfloat16_rn(v);
+    }
+    __syncthreads();
+    uint4* dst = reinterpret_cast<uint4*>(
+        out + (static_cast<size_t>(e) * per_expert + ti) * kTileBytes);
+    const uint4* src = reinterpret_cast<const uint4*>(tile);
+    for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads) dst[i] = src[i];
+}
+
 __global__ void amax_to_scale_kernel(float* scales, int n) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) scales[i] = fp8_scale_from_amax(__float_as_uint(scales[i]));
@@ -368,6 +424,29 @@ cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, co
         pack_tiles_kernel<false, false><<<gdn, kThreads, 0, s>>>(d, nullptr, H, I, geo.mt_dn,
                                                                  geo.kb_dn, dn, nullptr);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_lora(int E, int H, int I, int n_adapters, int rank, const void* Ag,
+                             const void* Bg, const void* Au, const void* Bu, const void* Ad,
+                             const void* Bd, void* packed, cudaStream_t s) {
+    const LoraGeom lg = lora_geom(E, H, I);
+    const int R = n_adapters * rank;
+    const auto* ag = static_cast<const __nv_bfloat16*>(Ag);
+    const auto* bg = static_cast<const __nv_bfloat16*>(Bg);
+    const auto* au = static_cast<const __nv_bfloat16*>(Au);
+    const auto* bu = static_cast<const __nv_bfloat16*>(Bu);
+    const auto* ad = static_cast<const __nv_bfloat16*>(Ad);
+    const auto* bd = static_cast<const __nv_bfloat16*>(Bd);
+    uint8_t* base = static_cast<uint8_t*>(packed);
+    pack_lora_kernel<0><<<dim3(lg.kb_gu, 1, E), kThreads, 0, s>>>(
+        ag, bg, au, bu, ad, bd, E, H, I, rank, R, lg.kb_gu, base + lg.shrink_gu);
+    pack_lora_kernel<1><<<dim3(lg.mt_gu * 2, 1, E), kThreads, 0, s>>>(
+        ag, bg, au, bu, ad, bd, E, H, I, rank, R, lg.mt_gu * 2, base + lg.expand_gu);
+    pack_lora_kernel<2><<<dim3(lg.kb_dn, 1, E), kThreads, 0, s>>>(
+        ag, bg, au, bu, ad, bd, E, H, I, rank, R, lg.kb_dn, base + lg.shrink_d);
+    pack_lora_kernel<3><<<dim3(lg.mt_dn, 1, E), kThreads, 0, s>>>(
+        ag, bg, au, bu, ad, bd, E, H, I, rank, R, lg.mt_dn, base + lg.expand_d);
     return cudaGetLastError();
 }
 

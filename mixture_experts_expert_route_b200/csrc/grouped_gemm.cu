@@ -87,8 +87,24 @@ constexpr int kStagingBytes = 16 * 1024;   // 2 KB per epilogue warp
 constexpr int kSmemCap = 232448;     // per-block opt-in limit on sm_100
 constexpr uint64_t kDrainLimitNs = 10000000ull;  // 10 ms
 
+// Tensor maps of one launch: weight tiles (pairs), activation rows, and the
+// adapters' expand tiles and shrink-output rows (multi-LoRA layers).
+struct Maps {
+    CUtensorMap a;                 // weight tiles, boxes of KPS tiles (pairs)
+    CUtensorMap a1;                // weight tiles, one tile per box (pairs, adapters on)
+    CUtensorMap al;                // adapter expand tiles, one tile per box (pairs)
+    CUtensorMap b128, b64, b16;    // activation rows in permuted order
+    CUtensorMap l128, l64, l16;    // adapter shrink outputs (rows in permuted order)
+};
+
 struct GemmArgs {
     int E, Mw, K, KB, MT, MTu, Mvalid;   // MTu: weight tiles per unit step (MT, or pairs)
+    int KBm, KBx;              // k-blocks of the matrix, and of the adapters' expand
+                               // (KB = KBm + KBx)
+    const uint8_t* x_tiles;    // adapter expand tiles [E][MT][KBx] (KBx > 0)
+    const int32_t* adapter;    // shrink (EPI 3): adapter of each token, -1 = none
+    const float* lscale;       // shrink: scale of each adapter
+    int lrank, lR;             // shrink: rank r, and n_adapters * r
     int nmax, tmem_cols, stages;
     const uint8_t* a_tiles;
     int ldo;
@@ -252,6 +268,9 @@ __device__ __forceinline__ void raise_abort(Ctl& c, int32_t* status) {
 //   EPI 0: h = SiLU(gate) * up -> bf16 rows of h (permuted order)
 //   EPI 1: w * y -> bf16 rows of y_perm (permuted order)
 //   EPI 2: w * y added (fp32) into row `token` of the accumulator
+//   EPI 3: adapter shrink: output column c (c % 64 = a * r + q) belongs to
+//          adapter a; it keeps s_a * value for tokens of adapter a and 0 for
+//          every other token (treg holds the tokens' adapters) -> bf16 rows
 template <bool FP8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, int m_own, int c0,
                                                float (&v)[16], float sw, const float (&wreg)[8],
@@ -286,16 +305,27 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
                                       static_cast<long>(row) * g.ldo + col) = val;
         __syncwarp();
-    } else if constexpr (EPI == 1) {
+    } else if constexpr (EPI == 1 || EPI == 3) {
         __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(staging + ew * 1024);
+        if constexpr (EPI == 1) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float wi = __shfl_sync(kFull, wreg[i & 7], (c0 + i) >> 3);
-            st[i * 32 + lane] = __float2bfloat16_rn(v[i] * wi);
+            for (int i = 0; i < 16; ++i) {
+                const float wi = __shfl_sync(kFull, wreg[i & 7], (c0 + i) >> 3);
+                st[i * 32 + lane] = __float2bfloat16_rn(v[i] * wi);
+            }
+        } else {
+            const int slot = (m_own * kBM + 32 * q + lane) & 63;
+            const int ac = slot < g.lR ? slot / g.lrank : -2;   // this column's adapter
+            const float sc = ac >= 0 ? __ldg(g.lscale + ac) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int ai = __shfl_sync(kFull, treg[i & 7], (c0 + i) >> 3);
+                st[i * 32 + lane] = __float2bfloat16_rn(ai == ac ? v[i] * sc : 0.0f);
+            }
         }
         __syncwarp();
         const int hcol0 = m_own * kBM + 32 * q;
-        if (hcol0 < g.Mvalid) {
+        if (hcol0 < g.Mvalid && m_own < g.MT) {
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 const int piece = lane + 32 * t;
@@ -339,10 +369,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
 
 template <bool FP8, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB128,
-                        const __grid_constant__ CUtensorMap tmB64,
-                        const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
+    grouped_gemm_kernel(const __grid_constant__ Maps maps, const GemmArgs g) {
     // gate/up token rows: gathered by the kernel itself for one-CTA tiles;
     // CTA-pair tiles (large token tiles) read rows a gather kernel laid out
     // in permuted order, by TMA
@@ -425,11 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl.mma_issued = 0;
         }
         if (warp == 0 && lane == 0) {
-            if constexpr (PAIR) tma_prefetch_desc(&tmA);
+            if constexpr (PAIR) tma_prefetch_desc(g.KBx ? &maps.a1 : &maps.a);
             if constexpr (!GATHER) {
-                tma_prefetch_desc(&tmB128);
-                tma_prefetch_desc(&tmB64);
-                tma_prefetch_desc(&tmB16);
+                tma_prefetch_desc(&maps.b128);
+                tma_prefetch_desc(&maps.b64);
+                tma_prefetch_desc(&maps.b16);
             }
         }
         if (warp == kFwdWarp) {
@@ -509,51 +536,76 @@ __global__ void __launch_bounds__(kThreads, 1)
             // A pair loads full KPS-tile boxes of weights; a single CTA loads
             // exactly the stage's k-blocks.  The gate/up kernel's token rows
             // are not counted here: the gather warps deliver them.
-            auto stage_bytes = [&](const Seg& sg, int nk) -> uint32_t {
-                uint32_t b = 0;
-                if constexpr (!GATHER) {
-                    const int rows = PAIR ? sg.Nm / 2 : sg.N;
-                    const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
-                    b = static_cast<uint32_t>(nk * (n64 * 64 + n16 * 16) * kRowBytes);
-                }
-                return PAIR ? 2u * (static_cast<uint32_t>(KPS * kATileBytes) + b)
-                            : static_cast<uint32_t>(nk * kATileBytes) + b;
+            // (k-blocks past KBm are an adapter's expand: weights from the
+            // adapter tiles, rows from the shrink outputs, both by the
+            // producer; with adapters, weights are copied k-block by k-block)
+            auto stage_bytes = [&](const Seg& sg, int kb, int nk) -> uint32_t {
+                const int rows = PAIR ? sg.Nm / 2 : sg.N;
+                const int n64 = rows >> 6, n16 = (rows & 63) >> 4;
+                const uint32_t row_bytes = static_cast<uint32_t>((n64 * 64 + n16 * 16) * kRowBytes);
+                int nb = nk;   // k-blocks whose rows the producer copies
+                if constexpr (GATHER) nb = max(0, kb + nk - max(kb, g.KBm));
+                const uint32_t b = static_cast<uint32_t>(nb) * row_bytes;
+                const int na = (PAIR && g.KBx == 0) ? KPS : nk;
+                return (PAIR ? 2u : 1u) * (static_cast<uint32_t>(na * kATileBytes) + b);
             };
             auto load_a = [&](const Seg& sg, int kb, int nk, int st) {
                 int m_own = PAIR ? 2 * sg.m + rank : sg.m;
                 if (m_own > mt_last) m_own = mt_last;   // odd tile count: any valid tile
-                const size_t tile = (static_cast<size_t>(sg.e) * g.MT + m_own) * g.KB + kb;
-                if constexpr (PAIR)
-                    tma_load_2d_pair(smA + st * a_stage_bytes, &tmA, &ctl.full[st], 0,
-                                     static_cast<int>(tile * kTileRows), kEvictFirst);
-                else
-                    bulk_load(smA + st * a_stage_bytes, g.a_tiles + tile * kTileBytes,
-                              nk * kATileBytes, &ctl.full[st], kEvictFirst);
+                const size_t em = static_cast<size_t>(sg.e) * g.MT + m_own;
+                if (g.KBx == 0) {
+                    const size_t tile = em * g.KBm + kb;
+                    if constexpr (PAIR)
+                        tma_load_2d_pair(smA + st * a_stage_bytes, &maps.a, &ctl.full[st], 0,
+                                         static_cast<int>(tile * kTileRows), kEvictFirst);
+                    else
+                        bulk_load(smA + st * a_stage_bytes, g.a_tiles + tile * kTileBytes,
+                                  nk * kATileBytes, &ctl.full[st], kEvictFirst);
+                    return;
+                }
+                for (int q = 0; q < nk; ++q) {
+                    const int k = kb + q;
+                    const bool ext = k >= g.KBm;
+                    const size_t tile = ext ? em * g.KBx + (k - g.KBm) : em * g.KBm + k;
+                    uint8_t* dst = smA + st * a_stage_bytes + q * kATileBytes;
+                    if constexpr (PAIR)
+                        tma_load_2d_pair(dst, ext ? &maps.al : &maps.a1, &ctl.full[st], 0,
+                                         static_cast<int>(tile * kTileRows), kEvictFirst);
+                    else
+                        bulk_load(dst, (ext ? g.x_tiles : g.a_tiles) + tile * kTileBytes,
+                                  kATileBytes, &ctl.full[st], kEvictFirst);
+                }
             };
             auto load_b = [&](const Seg& sg, int kb, int nk, int st) {
                 const int rows = PAIR ? sg.Nm / 2 : sg.N;
                 const int n128 = rows >> 7, n64 = (rows & 127) >> 6, n16 = (rows & 63) >> 4;
                 for (int q = 0; q < nk; ++q) {
+                    const int k = kb + q;
+                    const bool ext = k >= g.KBm;
+                    if (GATHER && !ext) continue;   // the gather warps copy these rows
+                    const CUtensorMap* m128 = ext ? &maps.l128 : &maps.b128;
+                    const CUtensorMap* m64 = ext ? &maps.l64 : &maps.b64;
+                    const CUtensorMap* m16 = ext ? &maps.l16 : &maps.b16;
                     uint8_t* b = smB + st * b_stage_bytes + q * b_kb_bytes;
                     int row = sg.b_row + rank * rows;
-                    const int xk = (kb + q) * bk_elems;
+                    const int xk = ext ? (k - g.KBm) * 64 : k * bk_elems;
                     for (int j = 0; j < n128; ++j, row += 128, b += 128 * kRowBytes) {
                         if constexpr (PAIR)
-                            tma_load_2d_pair(b, &tmB128, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d_pair(b, m128, &ctl.full[st], xk, row, kEvictLast);
                         else
-                            tma_load_2d(b, &tmB128, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d(b, m128, &ctl.full[st], xk, row, kEvictLast);
                     }
                     for (int j = 0; j < n64; ++j, row += 64, b += 64 * kRowBytes) {
                         if constexpr (PAIR)
-                            tma_load_2d_pair(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d_pair(b, m64, &ctl.full[st], xk, row, kEvictLast);
                         else
-                            tma_load_2d(b, &tmB64, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d(b, m64, &ctl.full[st], xk, row, kEvictLast);
                     }
                     for (int j = 0; j < n16; ++j, row += 16, b += 16 * kRowBytes) {
                         if constexpr (PAIR)
-                            tma_load_2d_pair(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d_pair(b, m16, &ctl.full[st], xk, row, kEvictLast);
                         else
-                            tma_load_2d(b, &tmB16, &ctl.full[st], xk, row, kEvictLast);
+                            tma_load_2d(b, m16, &ctl.full[st], xk, row, kEvictLast);
                     }
                 }
             };
@@ -567,7 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const Seg sg = make_seg<PAIR>(ctl, g, u, kb0, kb1);
                     for (int kb = sg.kb0; kb < sg.kb1 && early < S; kb += KPS, ++early) {
                         const int nk = min(KPS, sg.kb1 - kb);
-                        if (rank == 0) mbar_arrive_expect_tx(&ctl.full[early], stage_bytes(sg, nk));
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(&ctl.full[early], stage_bytes(sg, kb, nk));
                         load_a(sg, kb, nk, early);
                     }
                 }
@@ -589,10 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        if (rank == 0) mbar_arrive_expect_tx(&ctl.full[st], stage_bytes(sg, nk));
+                        if (rank == 0) mbar_arrive_expect_tx(&ctl.full[st], stage_bytes(sg, kb, nk));
                         load_a(sg, kb, nk, st);
                     }
-                    if constexpr (!GATHER) load_b(sg, kb, nk, st);
+                    if (!GATHER || kb + nk > g.KBm) load_b(sg, kb, nk, st);
                     if (++st == S) {
                         st = 0;
                         par ^= 1u;
@@ -668,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    for (int q = 0; q < nk; ++q) {
+                    for (int q = 0; q < nk && kb + q < g.KBm; ++q) {
                         const long long kofs = static_cast<long long>(kb + q) * kRowBytes + c * 16;
                         const bool in_row = kofs < g.src_row_bytes;
                         const uint32_t dst0 = smB_u32 + st * b_stage_bytes + q * b_kb_bytes + cs;
@@ -854,8 +907,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         if (sid >= 0) {
-                            wreg[i] = __ldg(g.w + sid);
-                            treg[i] = sid / g.ktop;
+                            if constexpr (EPI == 3) {
+                                treg[i] = __ldg(g.adapter + sid / g.ktop);
+                            } else {
+                                wreg[i] = __ldg(g.w + sid);
+                                treg[i] = sid / g.ktop;
+                            }
                         }
                     }
                 }
@@ -1013,6 +1070,7 @@ constexpr int kMaxDevices = 64;
 
 template <bool FP8, int EPI, bool PAIR>
 cudaError_t opt_in_smem() {
+    static_assert(sizeof(Maps) % 64 == 0, "tensor maps are 64-byte aligned");
     static std::once_flag once[kMaxDevices];
     static cudaError_t err[kMaxDevices];
     int dev = 0;
@@ -1030,9 +1088,7 @@ cudaError_t opt_in_smem() {
 }
 
 template <bool FP8, int EPI, bool PAIR>
-cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b128, const CUtensorMap& b64,
-                     const CUtensorMap& b16, const GemmArgs& g, int grid, int smem,
-                     cudaStream_t s) {
+cudaError_t launch_t(const Maps& maps, const GemmArgs& g, int grid, int smem, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<FP8, EPI, PAIR>;
     const cudaError_t attr = opt_in_smem<FP8, EPI, PAIR>();
     if (attr != cudaSuccess) return attr;
@@ -1050,17 +1106,20 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b128, const CUtens
     at[1].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = PAIR ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, b128, b64, b16, g);
+    return cudaLaunchKernelEx(&cfg, kern, maps, g);
 }
 
 template <bool FP8, bool PAIR>
-cudaError_t launch_epi(int epi, const CUtensorMap& a, const CUtensorMap& b128,
-                       const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& g, int grid,
-                       int smem, cudaStream_t s) {
+cudaError_t launch_epi(int epi, const Maps& maps, const GemmArgs& g, int grid, int smem,
+                       cudaStream_t s) {
     switch (epi) {
-        case 0: return launch_t<FP8, 0, PAIR>(a, b128, b64, b16, g, grid, smem, s);
-        case 1: return launch_t<FP8, 1, PAIR>(a, b128, b64, b16, g, grid, smem, s);
-        default: return launch_t<FP8, 2, PAIR>(a, b128, b64, b16, g, grid, smem, s);
+        case 0: return launch_t<FP8, 0, PAIR>(maps, g, grid, smem, s);
+        case 1: return launch_t<FP8, 1, PAIR>(maps, g, grid, smem, s);
+        case 2: return launch_t<FP8, 2, PAIR>(maps, g, grid, smem, s);
+        default:
+            // the adapter shrink exists for bf16 layers only
+            if constexpr (FP8) return cudaErrorInvalidValue;
+            else return launch_t<FP8, 3, PAIR>(maps, g, grid, smem, s);
     }
 }
 
@@ -1105,8 +1164,15 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.K = p.K;
     g.Mvalid = p.Mvalid;
     g.nmax = p.nmax;
-    g.KB = p.KB;
+    g.KBm = p.KB;
+    g.KBx = p.KBx;
+    g.KB = p.KB + p.KBx;
     g.MT = p.MT;
+    g.x_tiles = static_cast<const uint8_t*>(p.x_tiles);
+    g.adapter = p.adapter;
+    g.lscale = p.lscale;
+    g.lrank = p.lrank;
+    g.lR = p.lR;
     // Large token tiles run on CTA pairs (M = 256 per MMA, each CTA loads
     // half of every token tile); weight streaming runs one CTA per SM.
     const bool pair = p.nmax > 64;
@@ -1149,28 +1215,41 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
         return cudaErrorInvalidValue;
     if (p.epi != 0 && (!p.sorted_ids || !p.w)) return cudaErrorInvalidValue;
     if (p.acc_zero_floats % 4 != 0) return cudaErrorInvalidValue;
-    CUtensorMap ta, tb128, tb64, tb16;
-    memset(&ta, 0, sizeof(ta));
-    memset(&tb128, 0, sizeof(tb128));
-    memset(&tb64, 0, sizeof(tb64));
-    memset(&tb16, 0, sizeof(tb16));
+    if (p.KBx > 0 && (p.fp8 || !p.x_tiles || !p.x_rows)) return cudaErrorInvalidValue;
+    if (p.epi == 3 && (p.fp8 || !p.adapter || !p.lscale || p.lrank < 1 || p.lR > 64))
+        return cudaErrorInvalidValue;
+    Maps maps;
+    memset(&maps, 0, sizeof(maps));
     // activation rows in permuted order come by TMA; a one-CTA gate/up
     // kernel gathers its rows itself and uses no activation maps
     const bool gathers = p.epi == 0 && !pair;
-    if (!gathers && (!p.act || !make_map(&tb128, p.act, p.fp8, p.K, p.capacity, 128) ||
-                     !make_map(&tb64, p.act, p.fp8, p.K, p.capacity, 64) ||
-                     !make_map(&tb16, p.act, p.fp8, p.K, p.capacity, 16)))
+    if (!gathers && (!p.act || !make_map(&maps.b128, p.act, p.fp8, p.K, p.capacity, 128) ||
+                     !make_map(&maps.b64, p.act, p.fp8, p.K, p.capacity, 64) ||
+                     !make_map(&maps.b16, p.act, p.fp8, p.K, p.capacity, 16)))
         return cudaErrorInvalidValue;
-    if (pair && !make_tile_map(&ta, p.weights, static_cast<long>(p.E) * p.MT * p.KB, kps))
-        return cudaErrorInvalidValue;
+    const long wtiles = static_cast<long>(p.E) * p.MT * p.KB;
+    if (pair && !make_tile_map(&maps.a, p.weights, wtiles, kps)) return cudaErrorInvalidValue;
+    if (p.KBx > 0) {
+        // adapter expand: rows of the shrink outputs (bf16, KBx * 64 wide)
+        // and, for pairs, both weight sources one tile per box
+        const int xk = p.KBx * 64;
+        if (!make_map(&maps.l128, p.x_rows, false, xk, p.capacity, 128) ||
+            !make_map(&maps.l64, p.x_rows, false, xk, p.capacity, 64) ||
+            !make_map(&maps.l16, p.x_rows, false, xk, p.capacity, 16))
+            return cudaErrorInvalidValue;
+        if (pair && (!make_tile_map(&maps.a1, p.weights, wtiles, 1) ||
+                     !make_tile_map(&maps.al, p.x_tiles,
+                                    static_cast<long>(p.E) * p.MT * p.KBx, 1)))
+            return cudaErrorInvalidValue;
+    }
     int grid = device_sm_count();
     if (p.max_ctas > 0 && p.max_ctas < grid) grid = p.max_ctas;
     if (pair) grid = grid < 2 ? 2 : grid & ~1;
     if (pair)
-        return p.fp8 ? launch_epi<true, true>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s)
-                     : launch_epi<false, true>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s);
-    return p.fp8 ? launch_epi<true, false>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s)
-                 : launch_epi<false, false>(p.epi, ta, tb128, tb64, tb16, g, grid, smem, s);
+        return p.fp8 ? launch_epi<true, true>(p.epi, maps, g, grid, smem, s)
+                     : launch_epi<false, true>(p.epi, maps, g, grid, smem, s);
+    return p.fp8 ? launch_epi<true, false>(p.epi, maps, g, grid, smem, s)
+                 : launch_epi<false, false>(p.epi, maps, g, grid, smem, s);
 }
 
 }  // namespace moe

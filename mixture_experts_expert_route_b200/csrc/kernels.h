@@ -36,6 +36,34 @@ inline PackedGeom packed_geom(int fp8, int E, int H, int I) {
     return g;
 }
 
+// Packed multi-LoRA adapters (bf16; n_adapters * rank = R <= 64), four
+// sections of 16 KB tiles in the same swizzled layout as the weights:
+//   shrink_gu [E][ceil(H/64)]   rows 0..63: A_g columns (row a*r+q), rows
+//                               64..127: A_u columns; K = H
+//   expand_gu [E][MT_gu][2]     per packed gate/up row (interleaved as W_gu):
+//                               k-block 0 = B_g (gate rows, else 0), k-block
+//                               1 = B_u (up rows, else 0); K index a*r+q
+//   shrink_d  [E][ceil(I/64)]   rows 0..R-1: A_d columns; K = I
+//   expand_d  [E][MT_dn][1]     per output column c: B_d[a][e][q][c]
+struct LoraGeom {
+    int kb_gu, kb_dn, mt_gu, mt_dn;
+    size_t shrink_gu, expand_gu, shrink_d, expand_d;   // byte offsets
+    size_t bytes;
+};
+inline LoraGeom lora_geom(int E, int H, int I) {
+    LoraGeom g;
+    g.kb_gu = (H + 63) / 64;
+    g.kb_dn = (I + 63) / 64;
+    g.mt_gu = (2 * I + kTileRows - 1) / kTileRows;
+    g.mt_dn = (H + kTileRows - 1) / kTileRows;
+    g.shrink_gu = 0;
+    g.expand_gu = g.shrink_gu + static_cast<size_t>(E) * g.kb_gu * kTileBytes;
+    g.shrink_d = g.expand_gu + static_cast<size_t>(E) * g.mt_gu * 2 * kTileBytes;
+    g.expand_d = g.shrink_d + static_cast<size_t>(E) * g.kb_dn * kTileBytes;
+    g.bytes = g.expand_d + static_cast<size_t>(E) * g.mt_dn * kTileBytes;
+    return g;
+}
+
 // Launch with programmatic dependent launch allowed (see pdl_wait/pdl_trigger).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -104,6 +132,9 @@ cudaError_t launch_pack_weights(int fp8, int E, int H, int I, const void* Wg, co
                                 const void* Wd, void* packed, float* scales, uint32_t* amax_tmp,
                                 cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(int32_t* status, int timeout_us, cudaStream_t s);
+cudaError_t launch_pack_lora(int E, int H, int I, int n_adapters, int rank, const void* Ag,
+                             const void* Bg, const void* Au, const void* Bu, const void* Ad,
+                             const void* Bd, void* packed, cudaStream_t s);
 
 // ---- a4/a6 (grouped_gemm.cu)
 struct GemmProblem {
@@ -111,6 +142,7 @@ struct GemmProblem {
     int epi;              // 0: gate/up, rows gathered from gather_src -> SiLU*up -> h
                           // 1: down -> * w -> bf16 rows of out (permuted order)
                           // 2: down -> * w -> added into fp32 row `token` of out
+                          // 3: adapter shrink -> masked, scaled bf16 rows of out
     int E, Mw, K;         // weight rows per expert, reduction length
     int Mvalid;           // weight rows per expert that are real (masking)
     int nmax;             // token-tile cap (multiple of 16, <= 256)
@@ -138,6 +170,16 @@ struct GemmProblem {
     int32_t* status;
     int max_ctas;
     int sched_after_wait;        // counts/offsets are written by the previous kernel
+    // multi-LoRA (bf16): the adapters' expand as KBx extra k-blocks of 64,
+    // weights from x_tiles [E][MT][KBx], rows from x_rows [capacity, KBx*64]
+    int KBx;
+    const void* x_tiles;
+    const void* x_rows;
+    // epi 3 (adapter shrink): the tokens' adapters, their scales, the rank,
+    // and n_adapters * rank (<= 64): output column c % 64 = a * rank + q
+    const int32_t* adapter;
+    const float* lscale;
+    int lrank, lR;
 };
 int gemm_nmax_for(int T, int k, int E);
 // Token tiles above 64 rows run on CTA pairs (whose gate/up rows are gathered

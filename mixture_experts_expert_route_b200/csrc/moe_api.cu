@@ -15,10 +15,14 @@ using namespace moe;
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kCtlInts = 640;  // status, amax_x, amax_h, counters (2 x kMaxCtas)
+// control block: status, amax_x, amax_h, stream-K counters of the gate/up and
+// down GEMMs and of the two adapter shrinks (kMaxCtas each)
+constexpr int kCtlInts = 64 + 4 * kMaxCtas;
 constexpr int kCtlStatus = 0, kCtlAmaxX = 1, kCtlAmaxH = 2, kCtlCountersGu = 64,
-              kCtlCountersDn = 64 + kMaxCtas;
-static_assert(kCtlCountersDn + kMaxCtas <= kCtlInts, "control block too small");
+              kCtlCountersDn = 64 + kMaxCtas, kCtlCountersSgu = 64 + 2 * kMaxCtas,
+              kCtlCountersSdn = 64 + 3 * kMaxCtas;
+// widths (bf16 columns) of the adapter shrink outputs: gate|up, and down
+constexpr int kLoraGuCols = 128, kLoraDnCols = 64;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -61,7 +65,10 @@ struct Carver {
 struct FfnBuffers {
     int32_t* ctl;
     void* xq;         // FP8: e4m3 codes of x, token order [T, H]
-    void* x_perm;     // CTA-pair tiles: permuted token rows [cap, H] (bf16 / e4m3)
+    void* x_perm;     // permuted token rows [cap, H] (bf16 / e4m3): CTA-pair tiles,
+                      // and every bf16 layer (adapters' shrink)
+    void* t_gu;       // adapters: shrink outputs of x [cap, 128] bf16
+    void* t_dn;       // adapters: shrink outputs of h [cap, 64] bf16
     void* h;
     void* h_q;
     float* partials;
@@ -71,8 +78,13 @@ void carve_ffn_rest(Carver& c, FfnBuffers& b, moe_dtype dt, int T, int cap, int 
                     int nmax) {
     const bool fp8 = dt == MOE_FP8_E4M3;
     b.xq = fp8 ? c.take<void>(static_cast<size_t>(T) * H) : nullptr;
-    b.x_perm = gemm_uses_pairs(nmax) ? c.take<void>(static_cast<size_t>(cap) * H * (fp8 ? 1 : 2))
-                                     : nullptr;
+    // bf16 layers always have room for permuted rows and the adapters'
+    // shrink outputs, so one workspace size serves calls with and without
+    b.x_perm = (gemm_uses_pairs(nmax) || !fp8)
+                   ? c.take<void>(static_cast<size_t>(cap) * H * (fp8 ? 1 : 2))
+                   : nullptr;
+    b.t_gu = fp8 ? nullptr : c.take<void>(static_cast<size_t>(cap) * kLoraGuCols * 2);
+    b.t_dn = fp8 ? nullptr : c.take<void>(static_cast<size_t>(cap) * kLoraDnCols * 2);
     b.h = c.take<void>(static_cast<size_t>(cap) * I * 2);
     b.h_q = fp8 ? c.take<void>(static_cast<size_t>(cap) * I) : nullptr;
     b.partials = c.take<float>(gemm_partials_bytes(nmax));
@@ -109,6 +121,7 @@ struct FfnCall {
     bool x_ready = false;        // FP8: amax(x) and the codes of x already written
     bool counts_from_prev = false;  // the permutation is the previous kernel's output
     Combine combine = Combine::kGatherSum;
+    const moe_lora_args* lora = nullptr;
 };
 
 void record(moe_event_t* ev, int i, cudaStream_t s) {
@@ -141,7 +154,10 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
         counts_from_prev = false;
     }
     const void* rows_src = fp8 ? b.xq : f.x;
-    if (gemm_uses_pairs(nmax)) {
+    const bool lora = f.lora != nullptr;
+    const LoraGeom lgeo = lora_geom(f.E, f.H, f.I);
+    const uint8_t* lpk = lora ? static_cast<const uint8_t*>(f.lora->packed) : nullptr;
+    if (gemm_uses_pairs(nmax) || lora) {
         // large token tiles: lay the token rows out in permuted order for
         // the pair GEMM's TMA loads
         Range r("moe: gather (a3)");
@@ -149,6 +165,40 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
                                f.cap, b.x_perm, s) != cudaSuccess)
             return MOE_ERR_CUDA;
         counts_from_prev = false;
+    }
+
+    // the adapters' shrink of x (all adapters, masked to the token's own)
+    GemmProblem shr{};
+    if (lora) {
+        shr.fp8 = 0;
+        shr.epi = 3;
+        shr.E = f.E;
+        shr.Mw = kTileRows;
+        shr.Mvalid = kLoraGuCols;
+        shr.K = f.H;
+        shr.nmax = nmax;
+        shr.capacity = f.cap;
+        shr.weights = lpk + lgeo.shrink_gu;
+        shr.MT = 1;
+        shr.KB = lgeo.kb_gu;
+        shr.act = b.x_perm;
+        shr.out = b.t_gu;
+        shr.ldo = kLoraGuCols;
+        shr.counts = f.counts;
+        shr.offsets = f.offsets;
+        shr.sorted_ids = f.sorted_ids;
+        shr.ktop = f.k;
+        shr.A = f.T * f.k;
+        shr.partials = b.partials;
+        shr.counters = b.ctl + kCtlCountersSgu;
+        shr.status = f.status;
+        shr.max_ctas = f.max_ctas;
+        shr.adapter = f.lora->adapter;
+        shr.lscale = f.lora->scale;
+        shr.lrank = f.lora->rank;
+        shr.lR = f.lora->n_adapters * f.lora->rank;
+        Range r("moe: adapter shrink of x");
+        if (launch_grouped_gemm(shr, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     record(ev, 2, s);
 
@@ -185,6 +235,11 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     gu.status = f.status;
     gu.max_ctas = f.max_ctas;
     gu.sched_after_wait = counts_from_prev ? 1 : 0;
+    if (lora) {
+        gu.KBx = kLoraGuCols / 64;
+        gu.x_tiles = lpk + lgeo.expand_gu;
+        gu.x_rows = b.t_gu;
+    }
     {
         Range r("moe: gate/up GEMM (a3 gather + a4)");
         if (launch_grouped_gemm(gu, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -196,6 +251,20 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
         if (launch_quant_rows_fp8(b.h, f.offsets, f.E, f.I, f.cap, amax_h, b.h_q, s) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
+    }
+    if (lora) {
+        // the adapters' shrink of h
+        GemmProblem sd = shr;
+        sd.Mvalid = kLoraDnCols;
+        sd.K = f.I;
+        sd.weights = lpk + lgeo.shrink_d;
+        sd.KB = lgeo.kb_dn;
+        sd.act = b.h;
+        sd.out = b.t_dn;
+        sd.ldo = kLoraDnCols;
+        sd.counters = b.ctl + kCtlCountersSdn;
+        Range r("moe: adapter shrink of h");
+        if (launch_grouped_gemm(sd, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     record(ev, 4, s);
 
@@ -217,6 +286,11 @@ moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaS
     dn.acc_zero = nullptr;
     dn.acc_zero_floats = 0;
     dn.counters = b.ctl + kCtlCountersDn;
+    if (lora) {
+        dn.KBx = kLoraDnCols / 64;
+        dn.x_tiles = lpk + lgeo.expand_d;
+        dn.x_rows = b.t_dn;
+    }
     dn.sched_after_wait = 0;   // the permutation is at least two kernels back
     {
         Range r(fused ? "moe: down GEMM + combine (a6 + a7)" : "moe: down GEMM (a6)");
@@ -365,6 +439,23 @@ moe_status moe_pack_weights(moe_dtype dtype, int E, int H, int I, const void* Wg
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_packed_lora_size(int E, int H, int I, int n_adapters, int rank) {
+    if (E < 1 || H < 64 || I < 64 || n_adapters < 1 || rank < 1) return 0;
+    if (n_adapters * rank > 64 || E > kMaxExperts || H % 64 || I % 64) return 0;
+    return lora_geom(E, H, I).bytes;
+}
+
+moe_status moe_pack_lora(int E, int H, int I, int n_adapters, int rank, const void* Ag,
+                         const void* Bg, const void* Au, const void* Bu, const void* Ad,
+                         const void* Bd, void* packed, moe_stream_t stream) {
+    if (E < 1 || H < 64 || I < 64 || n_adapters < 1 || rank < 1) return MOE_ERR_INVALID_ARG;
+    if (n_adapters * rank > 64 || E > kMaxExperts || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
+    if (!Ag || !Bg || !Au || !Bu || !Ad || !Bd || !packed || !aligned16(packed))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_pack_lora(E, H, I, n_adapters, rank, Ag, Bg, Au, Bu, Ad, Bd, packed,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t moe_grouped_ffn_workspace_size(moe_dtype dtype, int T, int k, int E, int H, int I,
                                       int block_m) {
     if (check_layer(dtype, T, k, E, H, I, block_m) != MOE_OK) return 0;
@@ -427,6 +518,14 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     if (a->max_ctas < 0) return MOE_ERR_INVALID_ARG;
     if (a->combine < MOE_COMBINE_AUTO || a->combine > MOE_COMBINE_FUSED)
         return MOE_ERR_INVALID_ARG;
+    if (a->lora) {
+        const moe_lora_args* l = a->lora;
+        if (a->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+        if (l->n_adapters < 1 || l->rank < 1) return MOE_ERR_INVALID_ARG;
+        if (l->n_adapters * l->rank > 64) return MOE_ERR_UNSUPPORTED;
+        if (a->T > 0 && (!l->adapter || !l->packed || !l->scale || !aligned16(l->packed)))
+            return MOE_ERR_INVALID_ARG;
+    }
     if (a->T == 0) return MOE_OK;
     if (!a->x || !a->logits || !a->packed || !a->out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(a->x) || !aligned16(a->packed) || !aligned16(a->out))
@@ -483,6 +582,7 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     // right before the gate/up GEMM, unless FP8 kernels come between
     f.counts_from_prev = permute_chunks(A) <= 1;
     f.combine = pick_combine(a->combine);
+    f.lora = a->lora;
     st = run_ffn(f, b.ffn, ev, s);
     if (st != MOE_OK) return st;
     {

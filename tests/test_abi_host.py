@@ -97,7 +97,7 @@ def test_argument_errors_return_synchronously(L):
 def _fwd(L, **kw):
     base = dict(dtype=0, T=4, k=2, E=8, H=256, I=512, block_m=16, x=0x1000, logits=0x1000,
                 packed=0x1000, scales=None, out=0x1000, ids=None, w=None, status=None,
-                max_ctas=0, events=None, n_events=0, combine=0)
+                max_ctas=0, events=None, n_events=0, combine=0, lora=None)
     base.update(kw)
     a = L._lib.ForwardArgs(*[base[f] for f, _ in L._lib.ForwardArgs._fields_])
     return a
@@ -122,6 +122,14 @@ def test_forward_argument_errors(L):
     assert call(_fwd(L, events=0x1000, n_events=3)) == INVALID
     assert call(_fwd(L, combine=3)) == INVALID                # unknown combine mode
     assert call(_fwd(L, combine=-1)) == INVALID
+    # adapters: bf16 only, n * r <= 64, pointers required
+    la = L._lib.LoraArgs(4, 16, 0x1000, 0x1000, 0x1000)
+    assert call(_fwd(L, lora=ctypes.pointer(la), dtype=1, scales=0x1000)) == UNSUP
+    assert call(_fwd(L, lora=ctypes.pointer(L._lib.LoraArgs(5, 16, 0x1000, 0x1000, 0x1000)))) == UNSUP
+    assert call(_fwd(L, lora=ctypes.pointer(L._lib.LoraArgs(0, 16, 0x1000, 0x1000, 0x1000)))) == INVALID
+    assert call(_fwd(L, lora=ctypes.pointer(L._lib.LoraArgs(4, 16, None, 0x1000, 0x1000)))) == INVALID
+    assert lib.moe_packed_lora_size(8, 256, 512, 4, 16) > 0
+    assert lib.moe_packed_lora_size(8, 256, 512, 4, 17) == 0
     assert call(_fwd(L), 64) == WS                            # workspace too small
     assert call(_fwd(L, T=0, x=None, logits=None)) == 0       # T = 0 no-op
     assert lib.moe_forward(None, ws, big, None) == INVALID
