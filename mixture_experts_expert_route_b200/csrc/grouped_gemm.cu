@@ -1213,7 +1213,8 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     g.sched_after_wait = p.sched_after_wait ? 1 : 0;
     if (p.epi == 0 && !pair && (!p.gather_src || !p.sorted_ids || p.ktop < 1))
         return cudaErrorInvalidValue;
-    if (p.epi != 0 && (!p.sorted_ids || !p.w)) return cudaErrorInvalidValue;
+    if ((p.epi == 1 || p.epi == 2) && (!p.sorted_ids || !p.w)) return cudaErrorInvalidValue;
+    if (p.epi == 3 && !p.sorted_ids) return cudaErrorInvalidValue;
     if (p.acc_zero_floats % 4 != 0) return cudaErrorInvalidValue;
     if (p.KBx > 0 && (p.fp8 || !p.x_tiles || !p.x_rows)) return cudaErrorInvalidValue;
     if (p.epi == 3 && (p.fp8 || !p.adapter || !p.lscale || p.lrank < 1 || p.lR > 64))

@@ -73,8 +73,10 @@ def test_lora_stream_k_splits(moe, max_ctas):
 
 
 def test_lora_all_base_tokens_equal_base_layer(moe):
-    """Every token on the base model (-1): bit-identical to the layer without
-    adapters (the masked shrink outputs are zero, so the expand adds 0)."""
+    """Every token on the base model (-1): the masked shrink outputs are zero,
+    so the expand adds exact zeros; the result matches the layer without
+    adapters up to the fp32 summation grouping (the two extra k-blocks move
+    the stream-K split points), and the base oracle."""
     L = make_layer("tiny", T=50, E=8, k=2, H=256, I=256, seed=3)
     lora = make_lora(8, 256, 256, n_adapters=4, rank=16, seed=3)
     ad = torch.full((50,), -1, dtype=torch.int32)
@@ -83,7 +85,10 @@ def test_lora_all_base_tokens_equal_base_layer(moe):
     packed, _ = moe.pack_weights(moe.BF16, Wg, Wu, Wd)
     plain = moe.forward(moe.BF16, L.x.to(DEV), L.logits.to(DEV), packed, None, 8, 256, 2)
     torch.cuda.synchronize()
-    assert torch.equal(out, plain)
+    diff = (out.float() - plain.float()).abs().max().item()
+    assert diff <= 2 ** -7 * plain.float().abs().max().item()
+    ids_o, w_o = oracle.route_topk(L.logits, 2)
+    assert_close(out, oracle.moe_layer(L.x, ids_o, w_o, *L.weights_bf16()), 0, "lora, no adapter")
 
 
 def test_lora_prefill_shape(moe):
