@@ -48,6 +48,8 @@ WORKLOADS = {
     "prefill": dict(cfg="prefill", dtype=0, bound="tensor"),
     "fp8": dict(cfg="fp8", dtype=1, bound="tensor"),      # roofline entry at T=2048
     "skewed": dict(cfg="skewed", dtype=0, bound="tensor"),
+    # the prefill layer serving four rank-16 adapters (multi-LoRA)
+    "prefill_lora": dict(cfg="prefill", dtype=0, bound="tensor", lora=(4, 16)),
 }
 HEADLINE = "decode"
 NBATCH = 4
@@ -82,10 +84,12 @@ def traffic_for(workload, T):
 
 
 def describe(name):
-    c = CONFIGS[name]
-    d = "fp8 e4m3" if WORKLOADS[name]["dtype"] else "bf16"
+    wl = WORKLOADS[name]
+    c = CONFIGS[wl["cfg"]]
+    d = "fp8 e4m3" if wl["dtype"] else "bf16"
+    lo = f", {wl['lora'][0]} adapters of rank {wl['lora'][1]}" if wl.get("lora") else ""
     return (f"{name} {d} H={c['H']} I={c['I']} E={c['E']} top-{c['k']} "
-            f"T={','.join(str(t) for t in c['T'])}")
+            f"T={','.join(str(t) for t in c['T'])}{lo}")
 
 
 def gemm_token_cap(T, k, E):
@@ -97,7 +101,7 @@ def gemm_token_cap(T, k, E):
     return min(n, 256)
 
 
-def kernels_per_forward(T, k, E, fp8, H):
+def kernels_per_forward(T, k, E, fp8, H, lora=False):
     """Kernels one moe_forward launches."""
     A = T * k
     small = T <= SMALL_T and A <= CHUNK
@@ -107,7 +111,9 @@ def kernels_per_forward(T, k, E, fp8, H):
         n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
     # FP8: amax(x) and the codes of x (in the route kernel for small batches)
     n += 2 if fp8 and not (small and T * H <= SMALL_AMAX) else 0
-    n += 1 if gemm_token_cap(T, k, E) > 64 else 0   # gather (pair tiles; else in the GEMM)
+    # gather (pair tiles and adapter layers; else in the GEMM), adapter shrinks
+    n += 1 if gemm_token_cap(T, k, E) > 64 or lora else 0
+    n += 2 if lora else 0
     n += 1                                      # gate/up GEMM
     n += 1 if fp8 else 0                        # h quantisation
     n += 2                                      # down GEMM + combine (or finalize)
@@ -283,7 +289,7 @@ def cpu_baseline(W, dtype, T, budget_s, max_tokens=None, single_thread=True):
 # None = the whole batch).  The FP8 oracle runs whole batches (its h scale
 # needs every row), hence its small batch.
 ORACLE_SAMPLE = {"decode": (64, None), "prefill": (4096, 512), "fp8": (32, None),
-                 "skewed": (8192, 32)}
+                 "skewed": (8192, 32), "prefill_lora": (4096, 512)}
 
 
 def weight_device(name):
@@ -358,6 +364,15 @@ class Bench:
         Wg, Wu, Wd = (t.to(dev, torch.bfloat16) for t in (self.W.Wg, self.W.Wu, self.W.Wd))
         self.layer = moe.MoELayer(Wg, Wu, Wd, k=self.k, dtype=self.dtype)
         del Wg, Wu, Wd
+        self.lora, self.adapters = None, {}
+        if wl.get("lora"):
+            from workloads import adapter_ids, make_lora
+            n, r = wl["lora"]
+            lw = make_lora(self.E, self.H, self.I, n_adapters=n, rank=r, seed=1)
+            self.lora = moe.Lora(*(m.to(dev) for m in (lw.Ag, lw.Bg, lw.Au, lw.Bu, lw.Ad,
+                                                         lw.Bd)), lw.scale)
+            self.lora_rank = r
+            self.adapters = {T: adapter_ids(T, n, seed=T).to(dev) for T in self.Ts}
         self.batches = {T: [make_batch(self.W, T, 0, b) for b in range(NBATCH)]
                         for T in self.Ts}
         self.dev_in = {T: [(x.to(dev), lg.to(dev)) for x, lg in self.batches[T]]
@@ -388,13 +403,21 @@ class Bench:
         if self.layer.check() != 0:
             raise RuntimeError(f"{self.name}: device status word reports a fault")
 
+    def call(self, T, x, lg, out, ev=None):
+        if self.lora is None:
+            return self.layer(x, lg, out=out, events=ev)
+        return self.moe.forward(self.dtype, x, lg, self.layer.packed, self.layer.scales, self.E,
+                                self.I, self.k, out=out, status=self.layer.status,
+                                ws=self.layer.workspace(T), events=ev, lora=self.lora,
+                                adapter=self.adapters[T])
+
     def step(self, i, ev=None, direct=False):
         for T in self.Ts:
             if T in self.graphs and ev is None and not direct:
                 self.graphs[T][i % NBATCH].replay()
                 continue
             x, lg = self.dev_in[T][i % NBATCH]
-            self.layer(x, lg, out=self.outs[T], events=None if ev is None else ev[T])
+            self.call(T, x, lg, self.outs[T], ev=None if ev is None else ev[T])
 
     def capture_graphs(self):
         """Small token counts (T <= 64) run as CUDA graphs, one per rotating
@@ -411,7 +434,7 @@ class Bench:
                     x, lg = self.dev_in[T][b]
                     g = torch.cuda.CUDAGraph()
                     with torch.cuda.graph(g):
-                        self.layer(x, lg, out=self.outs[T])
+                        self.call(T, x, lg, self.outs[T])
                     gl.append(g)
                 self.graphs[T] = gl
             for i in range(self.args.warmup):
@@ -489,12 +512,12 @@ class Bench:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             x, lg = self.dev_in[T][0]
-            self.layer(x, lg, out=self.outs[T])
+            self.call(T, x, lg, self.outs[T])
             torch.cuda.synchronize()
             e0.record(self.stream)
             for i in range(args.steps):
                 x, lg = self.dev_in[T][i % NBATCH]
-                self.layer(x, lg, out=self.outs[T])
+                self.call(T, x, lg, self.outs[T])
             e1.record(self.stream)
             torch.cuda.synchronize()
             layer_direct_ms[T] = e0.elapsed_time(e1) / args.steps
@@ -539,6 +562,11 @@ class Bench:
             a = statistics.mean(self.active[T])
             layer_bytes = a * 3 * H * I * wb + T * H * 2 * 2 + T * E * 4
             layer_flops = 6.0 * T * k * H * I
+            if self.lora is not None:
+                # each assignment of an adapted token: shrink and expand of its
+                # own adapter on the three matrices (2r(H+I) MACs each)
+                n_ad = int((self.adapters[T] >= 0).sum().item())
+                layer_flops += 6.0 * n_ad * k * 2 * self.lora_rank * (H + I)
             lt = r["layer_graph_ms"].get(T, r["layer_direct_ms"][T])
             per_T[str(T)] = {
                 "layer_us": round(1e3 * lt, 2),
@@ -639,7 +667,8 @@ class Bench:
                           "double-buffered"}
 
     def launches(self):
-        return self.args.steps * sum(kernels_per_forward(T, self.k, self.E, self.fp8, self.H)
+        return self.args.steps * sum(kernels_per_forward(T, self.k, self.E, self.fp8, self.H,
+                                                         self.lora is not None)
                                      for T in self.Ts)
 
 
@@ -700,7 +729,7 @@ def run_native(args):
                    "dtype": "fp8" if wb.fp8 else "bf16", "roofline": rl, "per_T": pt,
                    "cuda_graphs": sorted(wb.graphs) if wb.graphs else (wb.graph_note or "none"),
                    "gpu_launches": wb.launches(), "clocks": c.summary()}
-            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and wb.lora is None:
                 T, pool = ORACLE_SAMPLE[name]
                 blk["cpu_baseline"] = cpu_baseline(wb.W, wb.dtype, T, args.cpu_seconds_other,
                                                    pool, single_thread=False)

@@ -81,6 +81,9 @@ def test_bench_mirrors_library_dispatch_constants():
     assert bench.kernels_per_forward(2048, 4, 32, True, 2880) == 11
     # prefill bf16 T=4096: route, 3 permutation kernels, gather, 2 GEMMs, finalize
     assert bench.kernels_per_forward(4096, 8, 128, False, 2048) == 8
+    # with adapters: the gather kernel and two shrink GEMMs more
+    assert bench.kernels_per_forward(4096, 8, 128, False, 2048, lora=True) == 10
+    assert bench.kernels_per_forward(1, 2, 8, False, 4096, lora=True) == 7
     # the token-tile cap (pair tiles above 64): twice the mean per expert
     assert bench.gemm_token_cap(64, 2, 8) == 32
     assert bench.gemm_token_cap(40, 2, 2) == 96
