@@ -74,7 +74,7 @@ namespace {
 constexpr int kBM = 128;            // weight rows per tile (UMMA M)
 constexpr int kRowBytes = 128;      // K bytes per stage row (one swizzle atom)
 constexpr int kATileBytes = kBM * kRowBytes;
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;         // at most; see threads_for
 constexpr int kFwdWarp = 2;           // TMEM allocator
 constexpr int kEpiWarp0 = 4;          // warps 4..11: two per TMEM lane quarter
 constexpr int kEpiThreads = 256;
@@ -367,8 +367,14 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const Seg& s, 
     }
 }
 
+// Threads of one instantiation: the gather warps (12-15) exist only where a
+// one-CTA gate/up kernel gathers its rows; the others run 384 threads, which
+// leaves more registers per thread for the epilogue.
+template <int EPI, bool PAIR>
+__host__ __device__ constexpr int threads_for() { return EPI == 0 && !PAIR ? 512 : 384; }
+
 template <bool FP8, int EPI, bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for<EPI, PAIR>(), 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const GemmArgs g) {
     // gate/up token rows: gathered by the kernel itself for one-CTA tiles;
     // CTA-pair tiles (large token tiles) read rows a gather kernel laid out
@@ -377,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int S = g.stages;
     // k-blocks per stage: 2 for a pair (large token tiles), 4 for one CTA
     constexpr int KPS = kps_for<PAIR>();
+    constexpr int NT = threads_for<EPI, PAIR>();
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ Ctl ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -471,18 +478,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         if (threadIdx.x == 0) {
             int run = 0;
-            for (int i = 0; i < kThreads / 32; ++i) {
+            for (int i = 0; i < NT / 32; ++i) {
                 const int t = ctl.scan_tmp[i];
                 ctl.scan_tmp[i] = run;
                 run += t;
             }
-            ctl.scan_tmp[kThreads / 32] = run;
+            ctl.scan_tmp[NT / 32] = run;
         }
         __syncthreads();
         if (e < g.E) ctl.full_prefix[e] = ctl.scan_tmp[warp] + inc - units;
         if (threadIdx.x == 0) {
-            ctl.full_prefix[g.E] = ctl.scan_tmp[kThreads / 32];
-            ctl.n_full_units = ctl.scan_tmp[kThreads / 32];
+            ctl.full_prefix[g.E] = ctl.scan_tmp[NT / 32];
+            ctl.n_full_units = ctl.scan_tmp[NT / 32];
         }
         // rank of e's partial tile among all partial tiles (keys are distinct)
         if (key != 0x7fffffff) {
@@ -496,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         if (threadIdx.x == 0) {
             int t = 0;
-            for (int i = 0; i < kThreads / 32; ++i) t += ctl.scan_tmp[i];
+            for (int i = 0; i < NT / 32; ++i) t += ctl.scan_tmp[i];
             ctl.n_partial = t;
         }
         tc_fence_before();
@@ -924,10 +931,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * g.nmax;
             if (s.kb0 == 0 && s.kb1 == g.KB) {
-                for (int c0 = 16 * half; c0 < s.N; c0 += 32) {
+                // this warp's chunks c0 and c0 + 32 loaded together, one wait
+                for (int c0 = 16 * half; c0 < s.N; c0 += 64) {
+                    const bool two = c0 + 32 < s.N;   // warp-uniform
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16_async(taddr + c0, r0);
+                    if (two) tmem_ld16_async(taddr + c0 + 32, r1);
+                    tmem_wait16(r0);
+                    if (two) tmem_wait16(r1);
                     float v[16];
-                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r0[i]);
                     epilogue_chunk<FP8, EPI>(g, s, m_own, c0, v, sw, wreg, treg, staging, amax);
+                    if (two) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r1[i]);
+                        epilogue_chunk<FP8, EPI>(g, s, m_own, c0 + 32, v, sw, wreg, treg, staging,
+                                                 amax);
+                    }
                 }
                 release(acc);
             } else {
@@ -1094,7 +1115,7 @@ cudaError_t launch_t(const Maps& maps, const GemmArgs& g, int grid, int smem, cu
     if (attr != cudaSuccess) return attr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads_for<EPI, PAIR>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute at[2];
