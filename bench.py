@@ -744,6 +744,31 @@ def run_native(args):
         dist.destroy_process_group()
 
 
+def run_calls(args):
+    """Profiling mode: N forward calls of one workload at one T (no timing, no
+    JSON), for a profiler to capture; the weights are drawn on the GPU."""
+    import mixture_experts_expert_route_b200 as moe
+    name = headline_name(args)
+    wl = WORKLOADS[name]
+    cfg = CONFIGS[wl["cfg"]]
+    T = int(args.Ts.split(",")[0]) if args.Ts else max(cfg["T"])
+    dev = torch.device("cuda", 0)
+    W = make_weights(wl["cfg"], 0, "cuda", E=args.experts)
+    layer = moe.MoELayer(W.Wg, W.Wu, W.Wd, k=cfg["k"], dtype=wl["dtype"])
+    E = W.E
+    del W
+    torch.cuda.empty_cache()
+    Wr = make_weights(wl["cfg"], 0, "cpu", E=args.experts, router_only=True)
+    x, lg = (t.to(dev) for t in make_batch(Wr, T, 0, 0))
+    out = torch.empty((T, cfg["H"]), dtype=torch.bfloat16, device=dev)
+    for _ in range(args.calls):
+        layer(x, lg, out=out)
+    torch.cuda.synchronize()
+    if layer.check() != 0:
+        raise RuntimeError("device status word reports a fault")
+    print(f"{name} T={T} E={E}: {args.calls} calls", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -764,7 +789,15 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--Ts", default="", help="comma-separated subset of the headline's "
                                             "token counts")
+    ap.add_argument("--calls", type=int, default=0,
+                    help="profiling mode: run this many forward calls of the workload (at the "
+                         "first of --Ts, else its largest T) and exit")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling mode: override the workload's expert count")
     args = ap.parse_args()
+    if args.calls > 0:
+        run_calls(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
