@@ -60,7 +60,25 @@ GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
 # while the sources still hash the same, and null (stale) otherwise.
 GEMM_SOURCES = ("mixture_experts_expert_route_b200/csrc/grouped_gemm.cu",
                 "mixture_experts_expert_route_b200/csrc/common.cuh")
-TRAFFIC = {}
+# DRAM bytes (read + write) of one gate/up launch, from ncu captures of the
+# committed profiling mode (`--calls 3`, cold cache), keyed by (workload, T);
+# each entry names the GEMM sources it was taken on and is reported only while
+# they are unchanged.  The skewed workload has none: only a scaled-down case
+# (E = 64, T = 1024) fits a capture, and its traffic does not scale to the
+# full workload in proportion to the units processed.
+TRAFFIC = {
+    ("decode", 64): {"bytes": 1886205440, "gemm_src": "6745066f5937",
+                     "capture": "profiles/grouped_gemm_decode_T64.md"},
+    ("prefill", 4096): {"bytes": 1377951232, "gemm_src": "6745066f5937",
+                        "capture": "profiles/grouped_gemm_prefill_T4096.md"},
+    ("fp8", 2048): {"bytes": 876110080, "gemm_src": "6745066f5937",
+                    "capture": "profiles/grouped_gemm_fp8_T2048.md"},
+}
+NO_TRAFFIC = {
+    "skewed": "not captured at full size (22.5 GB of weights); the scaled case E=64 T=1024 "
+              "(profiles/grouped_gemm_skewed_E64_T1024.md) does not scale in proportion",
+    "prefill_lora": "no ncu capture of the adapter variant",
+}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
 
@@ -77,7 +95,7 @@ def traffic_for(workload, T):
     """(bytes or None, note) for the roofline's `traffic` field."""
     rec = TRAFFIC.get((workload, T))
     if rec is None:
-        return None, "no ncu capture of this build"
+        return None, NO_TRAFFIC.get(workload, "no ncu capture of this build")
     if rec["gemm_src"] != gemm_source_hash():
         return None, f"stale: captured on GEMM sources {rec['gemm_src']} ({rec['capture']})"
     return rec["bytes"], f"ncu capture offline ({rec['capture']}), GEMM sources {rec['gemm_src']}"
