@@ -227,11 +227,18 @@ def test_combine_auto_is_deterministic(moe):
             assert diff <= 1e-2 * ref.float().abs().max().item()
 
 
+# FP8 paths of amax(x) and the codes of x: the single-CTA route kernel
+# (T = 24 / 48), and the amax and quantisation passes feeding one-CTA tiles
+# (T = 200, 64 experts) or the gather of CTA-pair tiles (T = 600, 4 experts)
+X_PATHS = [(24, 8), (200, 64), (600, 4)]
+
+
 @pytest.mark.parametrize("combine", COMBINES)
-def test_fp8_zero_input(moe, combine):
+@pytest.mark.parametrize("T,E", X_PATHS)
+def test_fp8_zero_input(moe, combine, T, E):
     """x = 0: amax = 0 gives s_x = 1 (and then h = 0, s_h = 1); the output is
     exactly zero, as the oracle's."""
-    L = make_layer("tiny", T=24, E=8, k=2, H=256, I=256, seed=3)
+    L = make_layer("tiny", T=T, E=E, k=2, H=256, I=256, seed=3)
     L.x = torch.zeros_like(L.x)
     out, ids, w = run_forward(moe, 1, L, combine=combine)
     ids_o, w_o = check_routing(ids, w, L.logits)
@@ -243,9 +250,10 @@ def test_fp8_zero_input(moe, combine):
 
 # bf16 values a for which the fp32 product a * (1 / (a / 448)) rounds above
 # 448: the element equal to amax(x) must still get the largest code (448).
+@pytest.mark.parametrize("T,E", [(48, 8), (200, 64), (600, 4)])
 @pytest.mark.parametrize("amax", [8.1875, 11.25, 15.9375])
-def test_fp8_amax_element_saturates(moe, amax):
-    L = make_layer("tiny", T=48, E=8, k=2, H=256, I=256, seed=4)
+def test_fp8_amax_element_saturates(moe, amax, T, E):
+    L = make_layer("tiny", T=T, E=E, k=2, H=256, I=256, seed=4)
     x = L.x.clone()
     x[3, 17] = amax
     x[20, 200] = -amax
