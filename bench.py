@@ -53,7 +53,7 @@ WORKLOADS = {
 }
 HEADLINE = "decode"
 NBATCH = 4
-GRAPH_MAX_T = 64       # token counts that run as CUDA graphs
+GRAPH_MAX_T = 64       # token counts that --graphs runs as CUDA graphs
 # DRAM bytes (read + write) of one gate/up launch, from an ncu capture made
 # offline (profiles/), keyed by (workload, T).  Each value records the hash of
 # the GEMM's source files it was captured with; the bench reports it only
@@ -451,10 +451,12 @@ class Bench:
             self.call(T, x, lg, self.outs[T], ev=None if ev is None else ev[T])
 
     def capture_graphs(self):
-        """Small token counts (T <= 64) run as CUDA graphs, one per rotating
-        batch: there the layer is a short chain of short kernels and the launch
-        cost on the host would otherwise show.  Larger T launch directly."""
-        if self.args.no_graphs:
+        """With --graphs, small token counts (T <= 64) run as CUDA graphs, one
+        per rotating batch.  Off by default: measured on B200, the replays were
+        slower on the device than direct launches (decode T=1 128.1 vs 124.6 us,
+        FP8 T=1 52.2 vs 47.3 us; the layer is device-bound, and the direct
+        chain keeps more of the programmatic-launch overlap)."""
+        if not self.args.graphs:
             return
         try:
             for T in self.Ts:
@@ -821,8 +823,11 @@ def main():
                     help="all: decode headline plus a block per other workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graphs", action="store_true",
+                    help="run T <= 64 as CUDA graph replays (default: direct launches, which "
+                         "measured faster on the device)")
     ap.add_argument("--no-graphs", action="store_true",
-                    help="launch every T directly (no CUDA graphs for T <= 64)")
+                    help="direct launches (the default; kept for older command lines)")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="oracle budget of the headline's CPU baseline (each of all-core "
                          "and single-thread)")
