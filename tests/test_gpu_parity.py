@@ -299,6 +299,48 @@ def test_nonfinite_logits(moe, dtype, combine):
     assert not torch.isfinite(out[9]).any()
 
 
+@pytest.mark.parametrize("T,E", X_PATHS)
+def test_fp8_nan_in_x(moe, T, E):
+    """A NaN element of x (reading R19): amax(x) skips it on both sides (a
+    maximum ignores NaN), it codes as NaN, and only its token's output is NaN;
+    every other token matches the oracle."""
+    L = make_layer("tiny", T=T, E=E, k=2, H=256, I=256, seed=12)
+    x = L.x.clone()
+    x[5, 10] = float("nan")
+    L.x = x
+    out, ids, w = run_forward(moe, 1, L)
+    ids_o, w_o = check_routing(ids, w, L.logits)
+    g, u, d = L.weights_bf16()
+    ref, _, (sx, _) = oracle.moe_layer_fp8(L.x, ids_o, w_o, g, u, d)
+    assert np.isfinite(sx)
+    assert np.isnan(ref).any(axis=1).tolist() == [t == 5 for t in range(T)]
+    assert np.isnan(ref[5]).all()
+    o = to_host(out).float()
+    assert torch.isnan(o[5]).all()
+    good = [t for t in range(T) if t != 5]
+    assert torch.isfinite(o[good]).all()
+    assert_close(out[good], ref[good], 1, f"NaN in x, T={T}")
+
+
+@pytest.mark.parametrize("T,E", X_PATHS)
+@pytest.mark.parametrize("val", [float("inf"), float("-inf")])
+def test_fp8_inf_in_x(moe, T, E, val):
+    """An infinite element of x (reading R19) makes amax(x) and s_x = amax/448
+    infinite; every finite element then codes as 0 and dequantises to
+    0 * inf = NaN, so the whole output is NaN, on both sides."""
+    L = make_layer("tiny", T=T, E=E, k=2, H=256, I=256, seed=13)
+    x = L.x.clone()
+    x[7, 3] = val
+    L.x = x
+    out, ids, w = run_forward(moe, 1, L)
+    ids_o, w_o = check_routing(ids, w, L.logits)
+    g, u, d = L.weights_bf16()
+    ref, _, (sx, _) = oracle.moe_layer_fp8(L.x, ids_o, w_o, g, u, d)
+    assert np.isinf(sx)
+    assert np.isnan(ref).all()
+    assert torch.isnan(to_host(out).float()).all()
+
+
 def test_forward_empty_batch(moe):
     L = make_layer("tiny", T=4, E=8, k=2, H=256, I=256)
     Wg, Wu, Wd = (W.to(DEV) for W in L.weights_bf16())
