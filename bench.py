@@ -67,11 +67,11 @@ GEMM_SOURCES = ("mixture_experts_expert_route_b200/csrc/grouped_gemm.cu",
 # (E = 64, T = 1024) fits a capture, and its traffic does not scale to the
 # full workload in proportion to the units processed.
 TRAFFIC = {
-    ("decode", 64): {"bytes": 1886205440, "gemm_src": "6745066f5937",
+    ("decode", 64): {"bytes": 1886205440, "gemm_src": "5b823d65316c",
                      "capture": "profiles/grouped_gemm_decode_T64.md"},
-    ("prefill", 4096): {"bytes": 1377951232, "gemm_src": "6745066f5937",
+    ("prefill", 4096): {"bytes": 1377951232, "gemm_src": "5b823d65316c",
                         "capture": "profiles/grouped_gemm_prefill_T4096.md"},
-    ("fp8", 2048): {"bytes": 876110080, "gemm_src": "6745066f5937",
+    ("fp8", 2048): {"bytes": 876110080, "gemm_src": "5b823d65316c",
                     "capture": "profiles/grouped_gemm_fp8_T2048.md"},
 }
 NO_TRAFFIC = {
@@ -83,11 +83,44 @@ SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
 
 
+def strip_comments(src):
+    """C/C++ source without comments, trailing blanks and empty lines (string
+    and character literals kept), so that the hash below follows the code."""
+    out, i, n, quote = [], 0, len(src), None
+    while i < n:
+        c = src[i]
+        if quote:
+            out.append(c)
+            if c == "\\" and i + 1 < n:
+                out.append(src[i + 1])
+                i += 2
+                continue
+            if c == quote:
+                quote = None
+            i += 1
+        elif c in "\"'":
+            quote = c
+            out.append(c)
+            i += 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(ln.rstrip() for ln in "".join(out).splitlines() if ln.strip())
+
+
 def gemm_source_hash():
+    """Hash of the GEMM's code (comments stripped): the key under which a
+    traffic capture stays valid."""
     h = hashlib.sha256()
     for p in GEMM_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p)) as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -29,11 +29,12 @@
 // kernel can add w * y into an fp32 accumulator in token order (the combine)
 // instead of writing permuted rows.
 //
-// Roles (512 threads): warp 0 = copy producer (weights; activation rows by
-// TMA where they are already in permuted order), warp 1 = MMA issuer (single
-// thread), warp 2 = TMEM allocator, warps 4-11 = epilogue (two warps per
-// 32-lane TMEM quarter, alternating 16-column chunks), warps 12-15 = gather of
-// a one-CTA gate/up kernel's token rows (cp.async).
+// Roles: warp 0 = copy producer (weights; activation rows by TMA where they
+// are already in permuted order), warp 1 = MMA issuer (single thread), warp 2
+// = TMEM allocator, warps 4-11 = epilogue (two warps per 32-lane TMEM quarter,
+// alternating 16-column chunks), and, in the one-CTA gate/up kernel only
+// (512 threads; the others run 384), warps 12-15 = gather of the token rows
+// (cp.async).
 // Shared-memory ring of stages of KPS k-blocks (A KPS*16 KB + B KPS*rows*128 B,
 // 128-byte swizzle): 2 stages of 4 k-blocks on one CTA (token tiles of at most
 // 64 rows), 3 stages of 2 k-blocks per CTA of a pair (larger tiles).  Two TMEM

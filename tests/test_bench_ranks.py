@@ -88,3 +88,15 @@ def test_bench_mirrors_library_dispatch_constants():
     assert bench.gemm_token_cap(64, 2, 8) == 32
     assert bench.gemm_token_cap(40, 2, 2) == 96
     assert bench.gemm_token_cap(4096, 8, 128) == 256
+
+
+def test_gemm_code_hash_ignores_comments_only():
+    """The traffic provenance key follows the code: comments and blank lines do
+    not change it, code does, and literals holding comment markers survive."""
+    import bench
+    src = 'int a = 1; // one\n/* block\n comment */ const char* s = "x // y /* z */";\n\nchar c = \'"\';\n'
+    same = 'int a = 1;   \n const char* s = "x // y /* z */"; // trailing\nchar c = \'"\'; /* c */\n'
+    assert bench.strip_comments(src) == bench.strip_comments(same)
+    assert '"x // y /* z */"' in bench.strip_comments(src)
+    assert bench.strip_comments(src) != bench.strip_comments(src.replace("a = 1", "a = 2"))
+    assert len(bench.gemm_source_hash()) == 12
