@@ -61,11 +61,10 @@ GRAPH_MAX_T = 64       # token counts that --graphs runs as CUDA graphs
 GEMM_SOURCES = ("mixture_experts_expert_route_b200/csrc/grouped_gemm.cu",
                 "mixture_experts_expert_route_b200/csrc/common.cuh")
 # DRAM bytes (read + write) of one gate/up launch, from ncu captures of the
-# committed profiling mode (`--calls 3`, cold cache), keyed by (workload, T);
-# each entry names the GEMM sources it was taken on and is reported only while
-# they are unchanged.  The skewed workload has none: only a scaled-down case
-# (E = 64, T = 1024) fits a capture, and its traffic does not scale to the
-# full workload in proportion to the units processed.
+# committed profiling mode (`--calls N`, cold cache), keyed by (workload, T);
+# each entry names the GEMM code it was taken on and is reported only while
+# that code is unchanged.  The full-size skewed launch is captured with the
+# three single-pass metrics only (duration, DRAM read and write bytes).
 TRAFFIC = {
     ("decode", 64): {"bytes": 1886205440, "gemm_src": "5b823d65316c",
                      "capture": "profiles/grouped_gemm_decode_T64.md"},
@@ -73,12 +72,12 @@ TRAFFIC = {
                         "capture": "profiles/grouped_gemm_prefill_T4096.md"},
     ("fp8", 2048): {"bytes": 876110080, "gemm_src": "5b823d65316c",
                     "capture": "profiles/grouped_gemm_fp8_T2048.md"},
+    ("skewed", 8192): {"bytes": 18309127168, "gemm_src": "5b823d65316c",
+                       "capture": "profiles/grouped_gemm_skewed_T8192.md"},
+    ("prefill_lora", 4096): {"bytes": 1461953536, "gemm_src": "5b823d65316c",
+                             "capture": "profiles/grouped_gemm_prefill_lora_T4096.md"},
 }
-NO_TRAFFIC = {
-    "skewed": "not captured at full size (22.5 GB of weights); the scaled case E=64 T=1024 "
-              "(profiles/grouped_gemm_skewed_E64_T1024.md) does not scale in proportion",
-    "prefill_lora": "no ncu capture of the adapter variant",
-}
+NO_TRAFFIC = {}
 SMALL_T, CHUNK = 128, 2048   # the library's single-CTA route+permute limits
 SMALL_AMAX = 32768           # x elements the single-CTA kernel also takes amax(x) of
 
@@ -838,8 +837,19 @@ def run_calls(args):
     Wr = make_weights(wl["cfg"], 0, "cpu", E=args.experts, router_only=True)
     x, lg = (t.to(dev) for t in make_batch(Wr, T, 0, 0))
     out = torch.empty((T, cfg["H"]), dtype=torch.bfloat16, device=dev)
+    call = lambda: layer(x, lg, out=out)
+    if wl.get("lora"):
+        # the adapter variant: the same adapters and token assignment as the bench
+        from workloads import adapter_ids, make_lora
+        n, r = wl["lora"]
+        lw = make_lora(E, cfg["H"], cfg["I"], n_adapters=n, rank=r, seed=1)
+        lora = moe.Lora(*(m.to(dev) for m in (lw.Ag, lw.Bg, lw.Au, lw.Bu, lw.Ad, lw.Bd)), lw.scale)
+        ad = adapter_ids(T, n, seed=T).to(dev)
+        call = lambda: moe.forward(wl["dtype"], x, lg, layer.packed, layer.scales, E, cfg["I"],
+                                   cfg["k"], out=out, status=layer.status, ws=layer.workspace(T),
+                                   lora=lora, adapter=ad)
     for _ in range(args.calls):
-        layer(x, lg, out=out)
+        call()
     torch.cuda.synchronize()
     if layer.check() != 0:
         raise RuntimeError("device status word reports a fault")
