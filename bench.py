@@ -380,6 +380,8 @@ def run_reference(args):
     if rank != 0:
         return
     name = headline_name(args)
+    if name == "split":
+        name = SPLIT["cfg"]     # the split computes the decode layer
     wl = WORKLOADS[name]
     # the same weights as the native arm (the skewed workload's 22.5 GB of
     # expert weights are drawn on the GPU there; the oracle copies the experts
@@ -747,6 +749,156 @@ class Bench:
                                      for T in self.Ts)
 
 
+# The CPU/GPU expert split (FIDDLER): the decode workload's experts
+# (Mixtral-8x7B-shaped) with half of them resident on the GPU (the ones a
+# profiling batch hits most), the others in host memory, run on the host or
+# copied to one of four staging slots per the measured latency model.
+SPLIT = dict(cfg="decode", budget=4, n_stage=4, profile_T=256)
+SPLIT_POLICIES = (("dynamic", 0), ("all_cpu", 1), ("all_staged", 2))
+
+
+def host_read_gbs(seconds=1.0):
+    """Host memory read bandwidth: a torch sum over 1 GiB of float32 on all
+    cores (the best of a few passes)."""
+    a = torch.ones(1 << 28, dtype=torch.float32)
+    best = 0.0
+    t_end = time.perf_counter() + seconds
+    while True:
+        t0 = time.perf_counter()
+        a.sum()
+        best = max(best, a.numel() * 4 / (time.perf_counter() - t0) / 1e9)
+        if time.perf_counter() > t_end:
+            break
+    del a
+    return best
+
+
+class SplitBench:
+    """moe_split_forward on the decode workload: per token count, the layer
+    under the dynamic plan and under the two fixed policies (every
+    non-resident expert on the host, or every one copied in)."""
+
+    def __init__(self, args, dev, Ts=None):
+        import mixture_experts_expert_route_b200 as moe
+        self.moe, self.args, self.dev = moe, args, dev
+        cfg = CONFIGS[SPLIT["cfg"]]
+        self.Ts = Ts or cfg["T"]
+        self.k, self.E, self.H, self.I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
+        W = make_weights(SPLIT["cfg"], 0, "cuda")
+        master = [t.cpu() for t in (W.Wg, W.Wu, W.Wd)]
+        W.Wg = W.Wu = W.Wd = None
+        torch.cuda.empty_cache()
+        self.W = W
+        # offline placement from a profiling batch's expert hits
+        xp, lp = make_batch(W, SPLIT["profile_T"], 1, 0)
+        ids, _ = moe.route_topk(lp.to(dev), self.k)
+        hits = torch.bincount(ids.flatten().long(), minlength=self.E).cpu().tolist()
+        self.resident = moe.split_place(hits, SPLIT["budget"])
+        self.layer = moe.SplitLayer(*master, self.k, self.resident, n_stage=SPLIT["n_stage"],
+                                    device=dev)
+        del master
+        self.dev_in = {T: [tuple(t.to(dev) for t in make_batch(W, T, 0, b))
+                           for b in range(NBATCH)] for T in self.Ts}
+        self.outs = {T: torch.empty((T, self.H), dtype=torch.bfloat16, device=dev)
+                     for T in self.Ts}
+
+    def measure(self, clk):
+        args, layer = self.args, self.layer
+        res = {}
+        expert_bytes = 3 * self.H * self.I * 2
+        clk.mark_start()
+        for T in self.Ts:
+            for pname, pol in SPLIT_POLICIES:
+                for i in range(args.warmup):
+                    x, lg = self.dev_in[T][i % NBATCH]
+                    layer(x, lg, out=self.outs[T], policy=pol)
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                places = {"resident": 0, "staged": 0, "cpu": 0}
+                e0.record()
+                for i in range(args.steps):
+                    x, lg = self.dev_in[T][i % NBATCH]
+                    layer(x, lg, out=self.outs[T], policy=pol)
+                    w = list(layer.where)
+                    places["resident"] += w.count(self.moe.SPLIT_RESIDENT)
+                    places["staged"] += w.count(self.moe.SPLIT_STAGED)
+                    places["cpu"] += w.count(self.moe.SPLIT_CPU)
+                e1.record()
+                torch.cuda.synchronize()
+                if layer.check() != 0:
+                    raise RuntimeError("split: device status word reports a fault")
+                ms = e0.elapsed_time(e1) / args.steps
+                mean = {key: v / args.steps for key, v in places.items()}
+                res[(T, pname)] = dict(ms=ms, places=mean,
+                                       bytes={key: v * expert_bytes for key, v in mean.items()})
+        clk.mark_end()
+        return res
+
+    def report(self, res, clocks):
+        hbm, _, src = peaks()
+        c = self.layer.costs
+        expert_bytes = 3 * self.H * self.I * 2
+        link = expert_bytes / (c.xfer_us * 1e-6) / 1e9           # GB/s, measured copy
+        host_bw = host_read_gbs()
+        per_T = {}
+        for T in self.Ts:
+            d = res[(T, "dynamic")]
+            b = d["bytes"]
+            # the host experts' weights stream from host memory while the GPU
+            # copies the staged ones over the link and streams the resident ones
+            ideal_ms = max(b["cpu"] / (host_bw * 1e9),
+                           b["staged"] / (link * 1e9) + (b["resident"] + b["staged"]) /
+                           (hbm * 1e9)) * 1e3
+            entry = {"layer_us": round(1e3 * d["ms"], 1),
+                     "tokens_per_s": round(T / (d["ms"] / 1e3), 1),
+                     "experts_per_call": {k2: round(v, 2) for k2, v in d["places"].items()},
+                     "ideal_us": round(1e3 * ideal_ms, 1),
+                     "frac_of_ideal": round(ideal_ms / d["ms"], 4)}
+            for pname, _ in SPLIT_POLICIES[1:]:
+                o = res[(T, pname)]
+                entry[f"{pname}_us"] = round(1e3 * o["ms"], 1)
+                entry[f"speedup_vs_{pname}"] = round(o["ms"] / d["ms"], 3)
+            per_T[str(T)] = entry
+        total_ms = sum(res[(T, "dynamic")]["ms"] for T in self.Ts)
+        return {"workload": f"split bf16 H={self.H} I={self.I} E={self.E} top-{self.k} "
+                            f"T={','.join(str(t) for t in self.Ts)}, "
+                            f"{SPLIT['budget']} experts resident, {SPLIT['n_stage']} staging slots",
+                "value": round(sum(self.Ts) / (total_ms / 1e3), 1), "unit": "tokens/s",
+                "ms_per_step": round(total_ms, 3), "dtype": "bf16",
+                "resident": [int(v) for v in self.resident],
+                "costs": {"cpu_us": round(c.cpu_us, 1),
+                          "cpu_us_per_token": round(c.cpu_us_per_token, 1),
+                          "xfer_us": round(c.xfer_us, 1), "gpu_us": c.gpu_us,
+                          "gpu_us_per_token": c.gpu_us_per_token},
+                "host_isa": "avx512_bf16" if self.moe.host_isa() else "portable",
+                "host_threads": os.cpu_count(), "cpu_model": cpu_model(),
+                "roofline": {"bound": "host memory | host link | hbm",
+                             "host_read_gbs": round(host_bw, 1),
+                             "link_h2d_gbs": round(link, 1), "hbm_gbs": hbm,
+                             "peak_source": src + " (HBM); host and link measured here",
+                             "note": "ideal = max(host experts' bytes / host read bandwidth, "
+                                     "staged bytes / link + GPU experts' bytes / HBM)"},
+                "per_T": per_T, "clocks": clocks,
+                "gpu_launches_per_call": "route, slot map, permute, gate/up + down per GPU "
+                                         "group, combine"}
+
+    def release(self):
+        del self.layer, self.dev_in, self.outs
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def run_split(args, dev, uuid):
+    c = ClockSampler(uuid).__enter__()
+    sb = SplitBench(args, dev)
+    r = sb.measure(c)
+    c.__exit__(None, None, None)
+    blk = sb.report(r, c.summary())
+    sb.release()
+    return blk
+
+
 def run_native(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -764,6 +916,14 @@ def run_native(args):
     atexit.register(clk.__exit__, None, None, None)   # stop the sampler on any exit path
     head = headline_name(args)
     Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else None
+    if head == "split":
+        clk.__exit__(None, None, None)
+        blk = run_split(args, dev, uuid)
+        if rank == 0:
+            print(json.dumps({"metric": "CPU/GPU split layer tokens/s", **blk,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "higher_is_better": True}), flush=True)
+        return
 
     b = Bench(head, args, dev, dist, world, Ts)
     r = b.measure(clk)
@@ -812,6 +972,9 @@ def run_native(args):
             wb.release()
             del wb
             blocks[name] = blk
+        if world == 1 and not args.no_split:
+            # host cores are shared by the ranks of one node: one GPU only
+            blocks["split"] = run_split(args, dev, uuid)
         line["workloads"] = blocks
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -862,7 +1025,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS), default="all",
+    ap.add_argument("--no-split", action="store_true",
+                    help="leave the CPU/GPU split block out of --workload all")
+    ap.add_argument("--workload", choices=["all", "split"] + sorted(WORKLOADS), default="all",
                     help="all: decode headline plus a block per other workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

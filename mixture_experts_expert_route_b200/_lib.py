@@ -55,6 +55,25 @@ class ForwardArgs(ctypes.Structure):
                 ("lora", ctypes.POINTER(LoraArgs))]
 
 
+class SplitCosts(ctypes.Structure):
+    _fields_ = [("cpu_us", ctypes.c_double), ("cpu_us_per_token", ctypes.c_double),
+                ("xfer_us", ctypes.c_double), ("gpu_us", ctypes.c_double),
+                ("gpu_us_per_token", ctypes.c_double)]
+
+
+class HostFfnArgs(ctypes.Structure):
+    _fields_ = [("H", I32), ("I", I32), ("n", I32), ("weights", P), ("x", P), ("w", P),
+                ("h", P), ("y", P), ("threads", I32), ("flags", I32)]
+
+
+class SplitArgs(ctypes.Structure):
+    _fields_ = [("T", I32), ("k", I32), ("E", I32), ("H", I32), ("I", I32), ("block_m", I32),
+                ("x", P), ("logits", P), ("out", P), ("resident", P), ("resident_packed", P),
+                ("stage_packed", P), ("n_stage", I32), ("host_packed", P), ("host_weights", P),
+                ("costs", ctypes.POINTER(SplitCosts)), ("policy", I32), ("where", P),
+                ("status", P), ("copy_stream", P), ("copy_event", P), ("host_threads", I32)]
+
+
 _SIGS = {
     "moe_status_string": ([I32], ctypes.c_char_p),
     "moe_version": ([], ctypes.c_char_p),
@@ -74,6 +93,18 @@ _SIGS = {
     "moe_forward": ([ctypes.POINTER(ForwardArgs), P, SZ, P], I32),
     "moe_check_status": ([P, P], I32),
     "moe_selftest_wait_timeout": ([P, I32, P], I32),
+    # CPU/GPU split (include/moe_split.h)
+    "moe_split_place": ([P, I32, I32, P], I32),
+    "moe_split_plan": ([P, P, I32, ctypes.POINTER(SplitCosts), I32, P], I32),
+    "moe_host_packed_size": ([I32, I32], SZ),
+    "moe_host_pack_weights": ([I32, I32, I32, P, P, P, P], I32),
+    "moe_host_isa": ([], I32),
+    "moe_host_expert_ffn": ([ctypes.POINTER(HostFfnArgs)], I32),
+    "moe_split_calibrate": ([I32, I32, I32, P, P, P, P, SZ, I32, P, ctypes.POINTER(SplitCosts)],
+                            I32),
+    "moe_split_workspace_size": ([I32, I32, I32, I32, I32, I32, I32, I32], SZ),
+    "moe_split_host_workspace_size": ([I32, I32, I32, I32], SZ),
+    "moe_split_forward": ([ctypes.POINTER(SplitArgs), P, SZ, P, SZ, P], I32),
 }
 
 _lib = None
@@ -325,6 +356,173 @@ class MoELayer:
                        self.k, out=out, status=self.status, ws=self.workspace(T),
                        block_m=self.block_m, max_ctas=self.max_ctas, events=events,
                        combine=self.combine, stream=stream)
+
+    def check(self) -> int:
+        return check_status(self.status)
+
+
+# ---- CPU/GPU expert split (include/moe_split.h) ----------------------------
+
+SPLIT_IDLE, SPLIT_RESIDENT, SPLIT_STAGED, SPLIT_CPU = 0, 1, 2, 3
+POLICY_DYNAMIC, POLICY_ALL_CPU, POLICY_ALL_STAGED = 0, 1, 2
+HOST_ISA_PORTABLE, HOST_ISA_AVX512_BF16 = 0, 1
+
+
+def _hptr(t):
+    """Address of a host (CPU) tensor or numpy array."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if t.is_cuda:
+            raise ValueError("expected a host tensor")
+        return t.data_ptr()
+    return t.ctypes.data
+
+
+def _i32(a):
+    import numpy as np
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def split_place(hits, budget: int):
+    """resident int32 [E]: 1 for the `budget` experts with the most hits."""
+    import numpy as np
+    h = np.ascontiguousarray(np.asarray(hits, dtype=np.int64))
+    resident = np.zeros(len(h), np.int32)
+    _check(lib().moe_split_place(_hptr(h), len(h), budget, _hptr(resident)), "moe_split_place")
+    return resident
+
+
+def split_costs(cpu_us=0.0, cpu_us_per_token=0.0, xfer_us=0.0, gpu_us=0.0,
+                gpu_us_per_token=0.0) -> SplitCosts:
+    return SplitCosts(cpu_us, cpu_us_per_token, xfer_us, gpu_us, gpu_us_per_token)
+
+
+def split_plan(counts, resident, costs: SplitCosts, n_stage: int):
+    """where int32 [E] (SPLIT_IDLE / RESIDENT / STAGED / CPU) for one batch."""
+    import numpy as np
+    c, r = _i32(counts), _i32(resident)
+    where = np.zeros(len(c), np.int32)
+    _check(lib().moe_split_plan(_hptr(c), _hptr(r), len(c), ctypes.byref(costs), n_stage,
+                                _hptr(where)), "moe_split_plan")
+    return where
+
+
+def host_isa() -> int:
+    return lib().moe_host_isa()
+
+
+def host_packed_size(H: int, I: int) -> int:
+    return lib().moe_host_packed_size(H, I)
+
+
+def host_pack_weights(Wg, Wu, Wd):
+    """Host layout of bf16 master weights (CPU tensors) -> uint8 CPU tensor [E, bytes]."""
+    E, H, I = Wg.shape
+    for W in (Wg, Wu, Wd):
+        if W.dtype != torch.bfloat16 or W.is_cuda or not W.is_contiguous():
+            raise ValueError("host master weights must be contiguous bf16 CPU tensors")
+    out = torch.empty((E, host_packed_size(H, I)), dtype=torch.uint8)
+    _check(lib().moe_host_pack_weights(E, H, I, _hptr(Wg), _hptr(Wu), _hptr(Wd), _hptr(out)),
+           "moe_host_pack_weights")
+    return out
+
+
+def host_expert_ffn(weights, x, w, threads: int = 0, portable: bool = False):
+    """One expert on the host: (h bf16 [n,I], y bf16 [n,H]).  weights: one row of
+    host_pack_weights' output; x bf16 [n,H]; w f32 [n] (CPU tensors)."""
+    n, H = x.shape
+    I = weights.numel() // (3 * H * 2)
+    x = x.contiguous()
+    w = w.to(torch.float32).contiguous()
+    h = torch.empty((n, I), dtype=torch.bfloat16)
+    y = torch.empty((n, H), dtype=torch.bfloat16)
+    a = HostFfnArgs(H, I, n, _hptr(weights), _hptr(x), _hptr(w), _hptr(h), _hptr(y), threads,
+                    1 if portable else 0)
+    _check(lib().moe_host_expert_ffn(ctypes.byref(a)), "moe_host_expert_ffn")
+    return h, y
+
+
+class SplitLayer:
+    """The CPU/GPU split layer (moe_split_forward): `resident` experts' weights
+    live on the GPU, the rest in host memory; each batch runs every other
+    expert it routes to either on the host or after copying its weights to
+    one of `n_stage` staging slots, as `policy` and `costs` decide.
+
+    Wg, Wu [E,H,I], Wd [E,I,H]: bf16 master weights on the host."""
+
+    def __init__(self, Wg, Wu, Wd, k: int, resident, n_stage: int = 2,
+                 policy: int = POLICY_DYNAMIC, costs: SplitCosts | None = None,
+                 host_threads: int = 0, block_m: int = 0, device="cuda"):
+        self.E, self.H, self.I = Wg.shape
+        self.k, self.n_stage, self.policy = k, n_stage, policy
+        self.host_threads, self.block_m = host_threads, block_m
+        self.device = torch.device(device)
+        self.resident = _i32(resident)
+        self.S = int(self.resident.sum())
+        E, H, I = self.E, self.H, self.I
+        self.host_weights = host_pack_weights(Wg, Wu, Wd)
+        # the GPU layout of all experts, made on the device once and kept in
+        # page-locked host memory as the source of the staging copies
+        pk, _ = pack_weights(BF16, Wg.to(self.device), Wu.to(self.device), Wd.to(self.device))
+        self.host_packed = torch.empty(pk.numel(), dtype=torch.uint8, pin_memory=True)
+        self.host_packed.copy_(pk)
+        del pk
+        idx = [e for e in range(E) if self.resident[e]]
+        self.resident_packed = None
+        if idx:
+            self.resident_packed, _ = pack_weights(BF16, Wg[idx].to(self.device),
+                                                   Wu[idx].to(self.device),
+                                                   Wd[idx].to(self.device))
+        self.stage_packed = torch.empty(
+            max(lib().moe_packed_weights_size(BF16, max(n_stage, 1), H, I), 16),
+            dtype=torch.uint8, device=self.device)
+        self.copy_stream = torch.cuda.Stream(device=self.device)
+        self.copy_event = torch.cuda.Event()
+        self.copy_event.record(self.copy_stream)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.where = _i32([0] * E)
+        self._ws, self._hws = {}, {}
+        self.costs = costs if costs is not None else self.calibrate()
+
+    def calibrate(self, n_max: int = 16) -> SplitCosts:
+        c = SplitCosts()
+        hws = torch.empty(lib().moe_split_host_workspace_size(n_max, 1, self.H, self.I),
+                          dtype=torch.uint8, pin_memory=True)
+        dst = self.stage_packed if self.n_stage > 0 else torch.empty(
+            3 * self.H * self.I * 2, dtype=torch.uint8, device=self.device)
+        _check(lib().moe_split_calibrate(self.H, self.I, n_max, _hptr(self.host_weights[0]),
+                                         _hptr(self.host_packed), _ptr(dst), _hptr(hws),
+                                         hws.numel(), self.host_threads, _stream(None),
+                                         ctypes.byref(c)), "moe_split_calibrate")
+        return c
+
+    def workspaces(self, T: int):
+        if T not in self._ws:
+            n = lib().moe_split_workspace_size(T, self.k, self.E, self.S, self.n_stage, self.H,
+                                               self.I, self.block_m)
+            if n == 0:
+                raise MoEError(1, "moe_split_workspace_size")
+            self._ws[T] = torch.empty(n, dtype=torch.uint8, device=self.device)
+            m = lib().moe_split_host_workspace_size(T, self.k, self.H, self.I)
+            self._hws[T] = torch.empty(max(m, 16), dtype=torch.uint8, pin_memory=True)
+        return self._ws[T], self._hws[T]
+
+    def __call__(self, x, logits, out=None, stream=None, policy: int | None = None):
+        T = x.shape[0]
+        out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device) \
+            if out is None else out
+        ws, hws = self.workspaces(T)
+        a = SplitArgs(T, self.k, self.E, self.H, self.I, self.block_m, _ptr(x), _ptr(logits),
+                      _ptr(out), _hptr(self.resident), _ptr(self.resident_packed),
+                      _ptr(self.stage_packed) if self.n_stage > 0 else None, self.n_stage,
+                      _hptr(self.host_packed), _hptr(self.host_weights),
+                      ctypes.pointer(self.costs), self.policy if policy is None else policy,
+                      _hptr(self.where), _ptr(self.status), self.copy_stream.cuda_stream,
+                      self.copy_event.cuda_event, self.host_threads)
+        _check(lib().moe_split_forward(ctypes.byref(a), _ptr(ws), ws.numel(), _hptr(hws),
+                                       hws.numel(), _stream(stream)), "moe_split_forward")
+        return out
 
     def check(self) -> int:
         return check_status(self.status)

@@ -17,7 +17,11 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["route_permute.cu", "elementwise.cu", "grouped_gemm.cu", "moe_api.cu", "noalloc.cu"]
+SOURCES = ["route_permute.cu", "elementwise.cu", "grouped_gemm.cu", "moe_api.cu", "noalloc.cu",
+           "split.cu"]
+# host code of the CPU/GPU split (g++: the AVX512_BF16 kernel selects its
+# instruction set per function and checks the CPU at run time)
+HOST_SOURCES = ["host_ffn.cpp"]
 HEADERS = ["common.cuh", "kernels.h"]
 LIB = os.path.join(HERE, "libmoe_b200.so")
 LIB_DEBUG = os.path.join(HERE, "libmoe_b200_debug.so")
@@ -39,8 +43,8 @@ def _stale(lib: str) -> bool:
     if not os.path.exists(lib):
         return True
     t = os.path.getmtime(lib)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
-    deps.append(os.path.join(ROOT, "include", "moe.h"))
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HOST_SOURCES + HEADERS]
+    deps += [os.path.join(ROOT, "include", h) for h in ("moe.h", "moe_split.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
@@ -61,8 +65,16 @@ def build(force: bool = False, ptxas_verbose: bool = False, debug: bool = False)
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         subprocess.check_call([nvcc(), *flags, "-c", os.path.join(CSRC, src), "-o", obj])
         objs.append(obj)
+    for src in HOST_SOURCES:
+        obj = os.path.join(objdir, src.replace(".cpp", ".o"))
+        subprocess.check_call(["g++", "-O3", "-std=c++17", "-fPIC", "-fvisibility=hidden",
+                               "-pthread", "-I", os.path.join(ROOT, "include"),
+                               *(["-DMOE_DEBUG_CHECKS"] if debug else []),
+                               "-c", os.path.join(CSRC, src), "-o", obj])
+        objs.append(obj)
     tmp = lib + f".{os.getpid()}.tmp"
-    subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"])
+    subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static",
+                           "-Xcompiler", "-pthread"])
     os.replace(tmp, lib)
     return lib
 

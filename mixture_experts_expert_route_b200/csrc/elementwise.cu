@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // a3 for large token tiles: dst[p] = src[sorted_ids[p] / k] for the rows
-// p < offsets[E] (pads zero), rows of vpr 16-byte vectors (bf16 x, or the
+// offsets[0] <= p < offsets[E] (pads zero), rows of vpr 16-byte vectors (bf16 x, or the
 // e4m3 codes of x).  One warp per row; each lane keeps up to 8 independent
 // 16-byte loads in flight before it stores them.
 __global__ void __launch_bounds__(kThreads)
@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(kThreads)
     const int lane = threadIdx.x & 31;
     const int rows = min(capacity, offsets[E]);
     const int wstride = gridDim.x * (kThreads / 32);
-    for (int p = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); p < rows; p += wstride) {
+    for (int p = offsets[0] + blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); p < rows;
+         p += wstride) {
         const int sid = sorted_ids[p];
         uint4* d = dst + static_cast<long>(p) * vpr;
         if (sid < 0) {

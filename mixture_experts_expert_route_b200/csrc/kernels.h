@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 // Packed expert weights are stored as 16 KB tiles, each the exact shared-memory
@@ -189,5 +191,17 @@ size_t gemm_partials_bytes(int nmax);
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 
 int device_sm_count();
+
+// ---- the bf16 grouped FFN (a3..a6) over E_sub consecutive segments of a
+// permutation (moe_api.cu): counts/offsets point at the first of them and
+// may start inside a larger permutation, whose other rows are left alone;
+// nmax is the token-tile cap (gemm_nmax_for of the segments' own mean).
+// Used by the CPU/GPU split, whose slot permutation spans several weight
+// buffers.  ws: segment_ffn_ws_bytes(T, capacity, H, I) bytes.
+size_t segment_ffn_ws_bytes(int T, int capacity, int H, int I);
+moe_status segment_ffn(int T, int k, int E_sub, int H, int I, int capacity, int nmax,
+                       const void* x, const float* w, const int32_t* counts,
+                       const int32_t* offsets, const int32_t* sorted_ids, const void* packed,
+                       void* y_perm, int32_t* status, void* ws, cudaStream_t s);
 
 }  // namespace moe

@@ -122,6 +122,7 @@ struct FfnCall {
     bool counts_from_prev = false;  // the permutation is the previous kernel's output
     Combine combine = Combine::kGatherSum;
     const moe_lora_args* lora = nullptr;
+    int nmax = 0;                   // token-tile cap; 0 = from T, k and E
 };
 
 void record(moe_event_t* ev, int i, cudaStream_t s) {
@@ -140,7 +141,7 @@ struct Range {
 // a3..a6 on carved buffers.  The control block must already be zeroed.
 moe_status run_ffn(const FfnCall& f, const FfnBuffers& b, moe_event_t* ev, cudaStream_t s) {
     const bool fp8 = f.dt == MOE_FP8_E4M3;
-    const int nmax = gemm_nmax_for(f.T, f.k, f.E);
+    const int nmax = f.nmax > 0 ? f.nmax : gemm_nmax_for(f.T, f.k, f.E);
     uint32_t* amax_x = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxX);
     uint32_t* amax_h = reinterpret_cast<uint32_t*>(b.ctl + kCtlAmaxH);
     const long x_elems = static_cast<long>(f.T) * f.H;
@@ -354,6 +355,32 @@ Combine pick_combine(int mode) {
 }
 
 }  // namespace
+
+namespace moe {
+
+size_t segment_ffn_ws_bytes(int T, int capacity, int H, int I) {
+    Carver c{nullptr};
+    carve_ffn(c, MOE_BF16, T, capacity, H, I, 256);   // partials for the largest cap
+    return c.used;
+}
+
+moe_status segment_ffn(int T, int k, int E_sub, int H, int I, int capacity, int nmax,
+                       const void* x, const float* w, const int32_t* counts,
+                       const int32_t* offsets, const int32_t* sorted_ids, const void* packed,
+                       void* y_perm, int32_t* status, void* ws, cudaStream_t s) {
+    if (E_sub < 1 || E_sub > kMaxExperts || nmax < 16 || nmax > 256) return MOE_ERR_INVALID_ARG;
+    Carver c{static_cast<char*>(ws)};
+    const FfnBuffers b = carve_ffn(c, MOE_BF16, T, capacity, H, I, 256);
+    if (cudaMemsetAsync(b.ctl, 0, sizeof(int32_t) * kCtlInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    FfnCall f{MOE_BF16, T, k, E_sub, H, I, capacity, x, w, counts, offsets, sorted_ids, packed,
+              nullptr, y_perm, status ? status : b.ctl + kCtlStatus, 0};
+    f.counts_from_prev = false;   // a memset comes between the permutation and the GEMM
+    f.nmax = nmax;
+    return run_ffn(f, b, nullptr, s);
+}
+
+}  // namespace moe
 
 extern "C" {
 
