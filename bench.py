@@ -752,9 +752,12 @@ class Bench:
 # The CPU/GPU expert split (FIDDLER): the decode workload's experts
 # (Mixtral-8x7B-shaped) with half of them resident on the GPU (the ones a
 # profiling batch hits most), the others in host memory, run on the host or
-# copied to one of four staging slots per the measured latency model.
-SPLIT = dict(cfg="decode", budget=4, n_stage=4, profile_T=256)
-SPLIT_POLICIES = (("dynamic", 0), ("all_cpu", 1), ("all_staged", 2))
+# copied to one of four staging slots per the measured latency model; decode
+# batches (T = 1..64) and prefill chunks (T = 512 and 2048, ~128 and ~512
+# tokens per expert).
+SPLIT = dict(cfg="decode", budget=4, n_stage=4, profile_T=256, T=(1, 4, 16, 64, 512, 2048))
+# "dynamic": the page's per-expert rule; "balanced": host and link in parallel
+SPLIT_POLICIES = (("dynamic", 0), ("balanced", 3), ("all_cpu", 1), ("all_staged", 2))
 
 
 def host_read_gbs(seconds=1.0):
@@ -782,7 +785,7 @@ class SplitBench:
         import mixture_experts_expert_route_b200 as moe
         self.moe, self.args, self.dev = moe, args, dev
         cfg = CONFIGS[SPLIT["cfg"]]
-        self.Ts = Ts or cfg["T"]
+        self.Ts = Ts or SPLIT["T"]
         self.k, self.E, self.H, self.I = cfg["k"], cfg["E"], cfg["H"], cfg["I"]
         W = make_weights(SPLIT["cfg"], 0, "cuda")
         master = [t.cpu() for t in (W.Wg, W.Wu, W.Wd)]
@@ -859,19 +862,31 @@ class SplitBench:
                 o = res[(T, pname)]
                 entry[f"{pname}_us"] = round(1e3 * o["ms"], 1)
                 entry[f"speedup_vs_{pname}"] = round(o["ms"] / d["ms"], 3)
+            bal = res[(T, "balanced")]
+            bb = bal["bytes"]
+            ideal_b = max(bb["cpu"] / (host_bw * 1e9),
+                          bb["staged"] / (link * 1e9) + (bb["resident"] + bb["staged"]) /
+                          (hbm * 1e9)) * 1e3
+            entry["balanced_experts_per_call"] = {k2: round(v, 2)
+                                                  for k2, v in bal["places"].items()}
+            entry["balanced_frac_of_ideal"] = round(ideal_b / bal["ms"], 4)
             per_T[str(T)] = entry
         total_ms = sum(res[(T, "dynamic")]["ms"] for T in self.Ts)
+        total_bal = sum(res[(T, "balanced")]["ms"] for T in self.Ts)
         return {"workload": f"split bf16 H={self.H} I={self.I} E={self.E} top-{self.k} "
                             f"T={','.join(str(t) for t in self.Ts)}, "
                             f"{SPLIT['budget']} experts resident, {SPLIT['n_stage']} staging slots",
                 "value": round(sum(self.Ts) / (total_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(total_ms, 3), "dtype": "bf16",
+                "policy": "dynamic (the per-expert rule); balanced_* fields: the host/link "
+                          "balanced plan",
+                "value_balanced": round(sum(self.Ts) / (total_bal / 1e3), 1),
                 "resident": [int(v) for v in self.resident],
                 "costs": {"cpu_us": round(c.cpu_us, 1),
                           "cpu_us_per_token": round(c.cpu_us_per_token, 1),
                           "xfer_us": round(c.xfer_us, 1), "gpu_us": c.gpu_us,
                           "gpu_us_per_token": c.gpu_us_per_token},
-                "host_isa": "avx512_bf16" if self.moe.host_isa() else "portable",
+                "host_isa": ["portable", "avx512_bf16", "amx_bf16"][self.moe.host_isa()],
                 "host_threads": os.cpu_count(), "cpu_model": cpu_model(),
                 "roofline": {"bound": "host memory | host link | hbm",
                              "host_read_gbs": round(host_bw, 1),
@@ -882,6 +897,25 @@ class SplitBench:
                 "per_T": per_T, "clocks": clocks,
                 "gpu_launches_per_call": "route, slot map, permute, gate/up + down per GPU "
                                          "group, combine"}
+
+    def host_kernel_rates(self, ns=(1, 16, 64, 128, 512)):
+        """moe_host_expert_ffn alone on expert 0 (all host threads, the best of
+        three runs per token count): weight bytes and FLOPs per second."""
+        H, I = self.H, self.I
+        out = {}
+        for n in ns:
+            x = torch.randn(n, H, generator=torch.Generator().manual_seed(n)).to(torch.bfloat16)
+            w = torch.ones(n)
+            self.moe.host_expert_ffn(self.layer.host_weights[0], x, w)
+            best = 1e9
+            for _ in range(3):
+                t0 = time.perf_counter()
+                self.moe.host_expert_ffn(self.layer.host_weights[0], x, w)
+                best = min(best, time.perf_counter() - t0)
+            out[str(n)] = {"ms": round(best * 1e3, 3),
+                           "weight_gbs": round(3 * H * I * 2 / best / 1e9, 1),
+                           "tflops": round(6.0 * n * H * I / best / 1e12, 2)}
+        return out
 
     def release(self):
         del self.layer, self.dev_in, self.outs
@@ -895,6 +929,7 @@ def run_split(args, dev, uuid):
     r = sb.measure(c)
     c.__exit__(None, None, None)
     blk = sb.report(r, c.summary())
+    blk["host_kernel"] = sb.host_kernel_rates()
     sb.release()
     return blk
 

@@ -13,7 +13,7 @@
  *     section: dynamic scheduling from token counts and expected latencies);
  *   - host experts run in a dedicated CPU kernel using AVX512_BF16 dot
  *     products where the CPU has them (same section, and § "2.先行研究との
- *     差別化ポイント").
+ *     差別化ポイント"); on CPUs with AMX, bf16 tile products.
  *
  * Everything else is the layer of moe.h: the GPU routes the batch, permutes
  * it by slot and runs the resident and copied experts in its grouped GEMMs;
@@ -42,8 +42,10 @@ typedef enum {
 typedef enum {
     MOE_SPLIT_POLICY_DYNAMIC = 0,   /* moe_split_plan with the given costs */
     MOE_SPLIT_POLICY_ALL_CPU = 1,   /* always the host */
-    MOE_SPLIT_POLICY_ALL_STAGED = 2 /* always copy the weights (while staging
+    MOE_SPLIT_POLICY_ALL_STAGED = 2,/* always copy the weights (while staging
                                        slots last; the rest on the host) */
+    MOE_SPLIT_POLICY_BALANCED = 3   /* moe_split_plan_balanced with the given
+                                       costs */
 } moe_split_policy;
 
 /*
@@ -86,6 +88,23 @@ MOE_API moe_status moe_split_plan(const int32_t* counts, const int32_t* resident
                                   const moe_split_costs* costs, int n_stage, int32_t* where);
 
 /*
+ * The balanced plan: the same latency model, with the host and the
+ * host-to-GPU link counted as two resources that work at the same time (an
+ * extension beyond the page, whose rule weighs each expert on its own).  The
+ * non-resident experts of a batch then cost
+ *   max( sum of cpu(n) over the experts left on the host,
+ *        sum of gpu(n) over the staged experts )
+ * Candidates (active, not resident) are ranked by cpu(n) / gpu(n), largest
+ * first (gpu(n) <= 0 first; equal ratios: lower index first), and the first
+ * j of them are staged, j in 0..min(n_stage, #candidates) minimising that
+ * maximum (equal maxima: the smaller j).  Sums run in rank order.  Arguments
+ * and errors as moe_split_plan.
+ */
+MOE_API moe_status moe_split_plan_balanced(const int32_t* counts, const int32_t* resident,
+                                           int E, const moe_split_costs* costs, int n_stage,
+                                           int32_t* where);
+
+/*
  * Host expert weights.  moe_host_pack_weights converts host bf16 master
  * weights W_g, W_u [E,H,I] and W_d [E,I,H] (row-major, as for
  * moe_pack_weights) into the host kernel's layout: per expert a block of
@@ -100,8 +119,10 @@ MOE_API size_t moe_host_packed_size(int H, int I);
 MOE_API moe_status moe_host_pack_weights(int E, int H, int I, const uint16_t* Wg,
                                          const uint16_t* Wu, const uint16_t* Wd, void* packed);
 
-/* Instruction-set path the host kernel takes on this CPU. */
-enum { MOE_HOST_ISA_PORTABLE = 0, MOE_HOST_ISA_AVX512_BF16 = 1 };
+/* Instruction-set path the host kernel takes on this CPU: AMX bf16 tiles
+ * (where the CPU has them and the OS grants the process the tile state),
+ * else AVX512_BF16 pair dot products, else portable C++. */
+enum { MOE_HOST_ISA_PORTABLE = 0, MOE_HOST_ISA_AVX512_BF16 = 1, MOE_HOST_ISA_AMX_BF16 = 2 };
 MOE_API int moe_host_isa(void);
 
 /*
@@ -115,12 +136,13 @@ MOE_API int moe_host_isa(void);
  *   y        bf16 [n][H] (out)
  * threads: worker threads of the library's host pool to use (0 = all; the
  * pool has one thread per hardware thread and is created on first use).
- * flags: MOE_HOST_FLAG_PORTABLE takes the portable path even where
- * AVX512_BF16 is available.  Both paths sum in fp32; their results may
- * differ in the last bits (pair products summed in a different order).
+ * flags: MOE_HOST_FLAG_PORTABLE takes the portable path, MOE_HOST_FLAG_NO_AMX
+ * the AVX512_BF16 path, even where a faster one is available.  All paths sum
+ * in fp32; their results may differ in the last bits (products summed in a
+ * different order).
  * Errors: MOE_ERR_INVALID_ARG for bad sizes or NULL pointers.
  */
-enum { MOE_HOST_FLAG_PORTABLE = 1 };
+enum { MOE_HOST_FLAG_PORTABLE = 1, MOE_HOST_FLAG_NO_AMX = 2 };
 typedef struct {
     int H, I, n;
     const void* weights;
@@ -137,7 +159,8 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
 /*
  * The split layer, for one batch x [T,H], logits [T,E]:
  *   1. GPU: route (a1) into ids, w; copy ids, w and x to the host; wait.
- *   2. host: counts, then the plan (policy; moe_split_plan for DYNAMIC).
+ *   2. host: counts, then the plan (policy: moe_split_plan for DYNAMIC,
+ *      moe_split_plan_balanced for BALANCED).
  *   3. GPU: copy each STAGED expert's packed weights into a staging slot;
  *      map every assignment to a slot (0 = host, 1..S = the resident experts
  *      in ascending index, S+1.. = staged experts in ascending index) and
@@ -162,7 +185,7 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
  *                      moe_pack_weights layout of all E experts: the source
  *                      of the copies
  *   host_weights       host, moe_host_pack_weights layout of all E experts
- *   costs              latency model (DYNAMIC); may be NULL otherwise
+ *   costs              latency model (DYNAMIC, BALANCED); may be NULL otherwise
  *   where              optional host int32 [E] out: the plan that ran
  *   copy_stream, copy_event  optional: the weight copies run on copy_stream
  *                      and copy_event orders the staged FFN after them, so

@@ -96,6 +96,7 @@ _SIGS = {
     # CPU/GPU split (include/moe_split.h)
     "moe_split_place": ([P, I32, I32, P], I32),
     "moe_split_plan": ([P, P, I32, ctypes.POINTER(SplitCosts), I32, P], I32),
+    "moe_split_plan_balanced": ([P, P, I32, ctypes.POINTER(SplitCosts), I32, P], I32),
     "moe_host_packed_size": ([I32, I32], SZ),
     "moe_host_pack_weights": ([I32, I32, I32, P, P, P, P], I32),
     "moe_host_isa": ([], I32),
@@ -364,8 +365,9 @@ class MoELayer:
 # ---- CPU/GPU expert split (include/moe_split.h) ----------------------------
 
 SPLIT_IDLE, SPLIT_RESIDENT, SPLIT_STAGED, SPLIT_CPU = 0, 1, 2, 3
-POLICY_DYNAMIC, POLICY_ALL_CPU, POLICY_ALL_STAGED = 0, 1, 2
-HOST_ISA_PORTABLE, HOST_ISA_AVX512_BF16 = 0, 1
+POLICY_DYNAMIC, POLICY_ALL_CPU, POLICY_ALL_STAGED, POLICY_BALANCED = 0, 1, 2, 3
+HOST_ISA_PORTABLE, HOST_ISA_AVX512_BF16, HOST_ISA_AMX_BF16 = 0, 1, 2
+HOST_PATHS = {"auto": 0, "portable": 1, "avx512_bf16": 2}   # moe_host_ffn_args.flags
 
 
 def _hptr(t):
@@ -398,13 +400,15 @@ def split_costs(cpu_us=0.0, cpu_us_per_token=0.0, xfer_us=0.0, gpu_us=0.0,
     return SplitCosts(cpu_us, cpu_us_per_token, xfer_us, gpu_us, gpu_us_per_token)
 
 
-def split_plan(counts, resident, costs: SplitCosts, n_stage: int):
-    """where int32 [E] (SPLIT_IDLE / RESIDENT / STAGED / CPU) for one batch."""
+def split_plan(counts, resident, costs: SplitCosts, n_stage: int, balanced: bool = False):
+    """where int32 [E] (SPLIT_IDLE / RESIDENT / STAGED / CPU) for one batch:
+    the per-expert rule, or with ``balanced`` the host/link balanced plan."""
     import numpy as np
     c, r = _i32(counts), _i32(resident)
     where = np.zeros(len(c), np.int32)
-    _check(lib().moe_split_plan(_hptr(c), _hptr(r), len(c), ctypes.byref(costs), n_stage,
-                                _hptr(where)), "moe_split_plan")
+    fn = lib().moe_split_plan_balanced if balanced else lib().moe_split_plan
+    _check(fn(_hptr(c), _hptr(r), len(c), ctypes.byref(costs), n_stage, _hptr(where)),
+           "moe_split_plan")
     return where
 
 
@@ -428,9 +432,10 @@ def host_pack_weights(Wg, Wu, Wd):
     return out
 
 
-def host_expert_ffn(weights, x, w, threads: int = 0, portable: bool = False):
+def host_expert_ffn(weights, x, w, threads: int = 0, path: str = "auto"):
     """One expert on the host: (h bf16 [n,I], y bf16 [n,H]).  weights: one row of
-    host_pack_weights' output; x bf16 [n,H]; w f32 [n] (CPU tensors)."""
+    host_pack_weights' output; x bf16 [n,H]; w f32 [n] (CPU tensors).  path:
+    "auto" (the fastest this CPU has), "avx512_bf16" (no AMX) or "portable"."""
     n, H = x.shape
     I = weights.numel() // (3 * H * 2)
     x = x.contiguous()
@@ -438,7 +443,7 @@ def host_expert_ffn(weights, x, w, threads: int = 0, portable: bool = False):
     h = torch.empty((n, I), dtype=torch.bfloat16)
     y = torch.empty((n, H), dtype=torch.bfloat16)
     a = HostFfnArgs(H, I, n, _hptr(weights), _hptr(x), _hptr(w), _hptr(h), _hptr(y), threads,
-                    1 if portable else 0)
+                    HOST_PATHS[path])
     _check(lib().moe_host_expert_ffn(ctypes.byref(a)), "moe_host_expert_ffn")
     return h, y
 
@@ -485,7 +490,11 @@ class SplitLayer:
         self._ws, self._hws = {}, {}
         self.costs = costs if costs is not None else self.calibrate()
 
-    def calibrate(self, n_max: int = 16) -> SplitCosts:
+    def calibrate(self, n_max: int = 128) -> SplitCosts:
+        """The latency model measured here: the host kernel on 1 and n_max
+        tokens (a line through both: flat while the host streams weights,
+        steeper once its tile products bound it, so n_max sits where a copy
+        starts to compete) and one expert's copy to the GPU."""
         c = SplitCosts()
         hws = torch.empty(lib().moe_split_host_workspace_size(n_max, 1, self.H, self.I),
                           dtype=torch.uint8, pin_memory=True)

@@ -14,8 +14,14 @@
 //           over I, then y = bf16(w * .).
 // Decode batches give each host expert a handful of tokens, so the passes
 // are bound by the host's memory bandwidth: each weight block is read once
-// per group of eight tokens and stays in the core's cache for the next group.
+// per group of tokens and stays in the core's cache for the next group.
+// Where the CPU has AMX tiles the passes multiply 16 tokens x 32 K by 32 K x
+// 16 columns per tile instruction (the weight layout is already the tiles'
+// pair layout), which keeps them bound by memory up to hundreds of tokens;
+// otherwise eight tokens share each 64-byte AVX512_BF16 pair product.
 #include <immintrin.h>
+#include <sys/syscall.h>
+#include <unistd.h>
 
 #include <algorithm>
 #include <atomic>
@@ -24,6 +30,7 @@
 #include <cstdint>
 #include <cstring>
 #include <functional>
+#include <limits>
 #include <mutex>
 #include <thread>
 #include <vector>
@@ -277,6 +284,105 @@ MOE_AVX512BF16 void down_block_avx512(const uint16_t* D, int I, const uint16_t* 
     }
 }
 
+// ---- the same passes on AMX tiles.  TDPBF16PS adds A[M][32] (bf16, M token
+// rows) times B[16 pairs][16 columns] (bf16 pairs of consecutive K, one
+// 64-byte row per pair: a 1 KB slice of a weight block) into C[M][16] fp32.
+// Tiles: 0, 1 = C (gate, up; the down pass uses 0), 2 = A, 3, 4 = B.
+// (Measured on the GPU machine's 16-core host: sharing each weight tile between
+// two token blocks did not help at 128 tokens and slowed one token by 40%.)
+#define MOE_AMX __attribute__((target("amx-tile,amx-bf16,avx512f,avx512bw,avx512vl,avx512bf16")))
+
+struct alignas(64) TileConfig {
+    uint8_t palette;
+    uint8_t start_row;
+    uint8_t reserved[14];
+    uint16_t colsb[16];
+    uint8_t rows[16];
+};
+
+MOE_AMX void amx_config(int M) {
+    TileConfig cfg{};
+    cfg.palette = 1;
+    for (int t : {0, 1, 2}) {
+        cfg.rows[t] = static_cast<uint8_t>(M);
+        cfg.colsb[t] = 64;
+    }
+    for (int t : {3, 4}) {
+        cfg.rows[t] = 16;
+        cfg.colsb[t] = 64;
+    }
+    _tile_loadconfig(&cfg);
+}
+
+MOE_AMX void gate_up_block_amx(const uint16_t* G, const uint16_t* U, int H, const uint16_t* x,
+                               int n, int c, int I, uint16_t* h) {
+    const int hp = H / 2;
+    const uint16_t* g0 = G + static_cast<size_t>(c) * hp * kCols * 2;
+    const uint16_t* u0 = U + static_cast<size_t>(c) * hp * kCols * 2;
+    constexpr size_t kSlice = 16 * kCols * 2;   // elements of one 1 KB weight slice
+    alignas(64) float gv[16 * kCols], uv[16 * kCols];
+    for (int t0 = 0; t0 < n; t0 += 16) {
+        const int M = std::min(16, n - t0);
+        amx_config(M);
+        _tile_zero(0);
+        _tile_zero(1);
+        const uint16_t* xa = x + static_cast<size_t>(t0) * H;
+        for (int kk = 0; kk < H / 32; ++kk) {
+            _tile_loadd(2, xa + 32 * kk, H * 2);
+            _tile_loadd(3, g0 + kk * kSlice, 64);
+            _tile_loadd(4, u0 + kk * kSlice, 64);
+            _tile_dpbf16ps(0, 2, 3);
+            _tile_dpbf16ps(1, 2, 4);
+        }
+        _tile_stored(0, gv, 64);
+        _tile_stored(1, uv, 64);
+        _tile_release();
+        for (int t = 0; t < M; ++t) {
+            float* gr = gv + t * kCols;
+            for (int i = 0; i < kCols; ++i) gr[i] = silu(gr[i]) * uv[t * kCols + i];
+            store_bf16_16(h + static_cast<size_t>(t0 + t) * I + c * kCols, _mm512_load_ps(gr));
+        }
+    }
+}
+
+MOE_AMX void down_block_amx(const uint16_t* D, int I, const uint16_t* h, const float* w, int n,
+                            int c, int H, uint16_t* y) {
+    const int ip = I / 2;
+    const uint16_t* d0 = D + static_cast<size_t>(c) * ip * kCols * 2;
+    constexpr size_t kSlice = 16 * kCols * 2;
+    alignas(64) float yv[16 * kCols];
+    for (int t0 = 0; t0 < n; t0 += 16) {
+        const int M = std::min(16, n - t0);
+        amx_config(M);
+        _tile_zero(0);
+        const uint16_t* ha = h + static_cast<size_t>(t0) * I;
+        for (int kk = 0; kk < I / 32; ++kk) {
+            _tile_loadd(2, ha + 32 * kk, I * 2);
+            _tile_loadd(3, d0 + kk * kSlice, 64);
+            _tile_dpbf16ps(0, 2, 3);
+        }
+        _tile_stored(0, yv, 64);
+        _tile_release();
+        for (int t = 0; t < M; ++t)
+            store_bf16_16(y + static_cast<size_t>(t0 + t) * H + c * kCols,
+                          _mm512_mul_ps(_mm512_load_ps(yv + t * kCols),
+                                        _mm512_set1_ps(w[t0 + t])));
+    }
+}
+
+// AMX needs the CPU's tile instructions and, on Linux, the process's
+// permission to use the tile state (requested once).
+bool cpu_has_amx_bf16() {
+    static const bool has = [] {
+        if (!__builtin_cpu_supports("amx-tile") || !__builtin_cpu_supports("amx-bf16") ||
+            !__builtin_cpu_supports("avx512bf16"))
+            return false;
+        constexpr long kReqXcompPerm = 0x1023, kXfeatureXtiledata = 18;
+        return syscall(SYS_arch_prctl, kReqXcompPerm, kXfeatureXtiledata) == 0;
+    }();
+    return has;
+}
+
 bool cpu_has_avx512_bf16() {
     static const bool has = __builtin_cpu_supports("avx512f") &&
                             __builtin_cpu_supports("avx512bw") &&
@@ -337,6 +443,49 @@ moe_status moe_split_plan(const int32_t* counts, const int32_t* resident, int E,
     return MOE_OK;
 }
 
+moe_status moe_split_plan_balanced(const int32_t* counts, const int32_t* resident, int E,
+                                   const moe_split_costs* c, int n_stage, int32_t* where) {
+    if (!counts || !resident || !c || !where || E < 1 || E > 256 || n_stage < 0)
+        return MOE_ERR_INVALID_ARG;
+    struct Cand {
+        double ratio, cpu, gpu;
+        int e;
+    };
+    std::vector<Cand> cand;
+    for (int e = 0; e < E; ++e) {
+        if (counts[e] < 0) return MOE_ERR_INVALID_ARG;
+        if (counts[e] == 0) {
+            where[e] = MOE_SPLIT_IDLE;
+        } else if (resident[e]) {
+            where[e] = MOE_SPLIT_RESIDENT;
+        } else {
+            where[e] = MOE_SPLIT_CPU;
+            const double n = counts[e];
+            const double cpu = c->cpu_us + c->cpu_us_per_token * n;
+            const double gpu = c->xfer_us + c->gpu_us + c->gpu_us_per_token * n;
+            const double ratio = gpu <= 0 ? std::numeric_limits<double>::infinity() : cpu / gpu;
+            cand.push_back({ratio, cpu, gpu, e});
+        }
+    }
+    std::stable_sort(cand.begin(), cand.end(),
+                     [](const Cand& a, const Cand& b) { return a.ratio > b.ratio; });
+    const int m = std::min<int>(n_stage, static_cast<int>(cand.size()));
+    int best_j = 0;
+    double best = 0;
+    for (int j = 0; j <= m; ++j) {
+        double host = 0, link = 0;
+        for (size_t i = j; i < cand.size(); ++i) host += cand[i].cpu;
+        for (int i = 0; i < j; ++i) link += cand[i].gpu;
+        const double cost = std::max(host, link);
+        if (j == 0 || cost < best) {
+            best = cost;
+            best_j = j;
+        }
+    }
+    for (int i = 0; i < best_j; ++i) where[cand[i].e] = MOE_SPLIT_STAGED;
+    return MOE_OK;
+}
+
 size_t moe_host_packed_size(int H, int I) {
     if (!valid_dims(H, I)) return 0;
     return 3 * section_elems(H, I) * sizeof(uint16_t);
@@ -358,6 +507,7 @@ moe_status moe_host_pack_weights(int E, int H, int I, const uint16_t* Wg, const 
 }
 
 int moe_host_isa(void) {
+    if (cpu_has_amx_bf16()) return MOE_HOST_ISA_AMX_BF16;
     return cpu_has_avx512_bf16() ? MOE_HOST_ISA_AVX512_BF16 : MOE_HOST_ISA_PORTABLE;
 }
 
@@ -370,13 +520,20 @@ moe_status moe_host_expert_ffn(const moe_host_ffn_args* a) {
     const uint16_t* G = static_cast<const uint16_t*>(a->weights);
     const uint16_t* U = G + m;
     const uint16_t* D = U + m;
-    const bool fast = cpu_has_avx512_bf16() && !(a->flags & MOE_HOST_FLAG_PORTABLE);
+    const bool portable = (a->flags & MOE_HOST_FLAG_PORTABLE) != 0;
+    const int isa = portable ? MOE_HOST_ISA_PORTABLE
+                    : (cpu_has_amx_bf16() && !(a->flags & MOE_HOST_FLAG_NO_AMX))
+                        ? MOE_HOST_ISA_AMX_BF16
+                        : cpu_has_avx512_bf16() ? MOE_HOST_ISA_AVX512_BF16
+                                                : MOE_HOST_ISA_PORTABLE;
     pool().run(I / kCols, a->threads, [&](int c) {
-        if (fast) gate_up_block_avx512(G, U, H, a->x, n, c, I, a->h);
+        if (isa == MOE_HOST_ISA_AMX_BF16) gate_up_block_amx(G, U, H, a->x, n, c, I, a->h);
+        else if (isa == MOE_HOST_ISA_AVX512_BF16) gate_up_block_avx512(G, U, H, a->x, n, c, I, a->h);
         else gate_up_block_portable(G, U, H, a->x, n, c, I, a->h);
     });
     pool().run(H / kCols, a->threads, [&](int c) {
-        if (fast) down_block_avx512(D, I, a->h, a->w, n, c, H, a->y);
+        if (isa == MOE_HOST_ISA_AMX_BF16) down_block_amx(D, I, a->h, a->w, n, c, H, a->y);
+        else if (isa == MOE_HOST_ISA_AVX512_BF16) down_block_avx512(D, I, a->h, a->w, n, c, H, a->y);
         else down_block_portable(D, I, a->h, a->w, n, c, H, a->y);
     });
     return MOE_OK;

@@ -224,9 +224,11 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     const int T = a->T, k = a->k, E = a->E, H = a->H, I = a->I;
     if (!dims_ok(T, k, E, H, I, block_m)) return MOE_ERR_INVALID_ARG;
     if (!a->resident || a->n_stage < 0) return MOE_ERR_INVALID_ARG;
-    if (a->policy < MOE_SPLIT_POLICY_DYNAMIC || a->policy > MOE_SPLIT_POLICY_ALL_STAGED)
+    if (a->policy < MOE_SPLIT_POLICY_DYNAMIC || a->policy > MOE_SPLIT_POLICY_BALANCED)
         return MOE_ERR_INVALID_ARG;
-    if (a->policy == MOE_SPLIT_POLICY_DYNAMIC && !a->costs) return MOE_ERR_INVALID_ARG;
+    if ((a->policy == MOE_SPLIT_POLICY_DYNAMIC || a->policy == MOE_SPLIT_POLICY_BALANCED) &&
+        !a->costs)
+        return MOE_ERR_INVALID_ARG;
     if ((a->copy_stream == nullptr) != (a->copy_event == nullptr)) return MOE_ERR_INVALID_ARG;
     const int S = count_resident(a->resident, E);
     const int Es = 1 + S + a->n_stage;
@@ -276,6 +278,9 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     moe_status st;
     if (a->policy == MOE_SPLIT_POLICY_DYNAMIC) {
         st = moe_split_plan(counts.data(), a->resident, E, a->costs, a->n_stage, where.data());
+    } else if (a->policy == MOE_SPLIT_POLICY_BALANCED) {
+        st = moe_split_plan_balanced(counts.data(), a->resident, E, a->costs, a->n_stage,
+                                     where.data());
     } else {
         // ALL_CPU: no expert gains from a copy; ALL_STAGED: every one does
         // (equal savings, so staging slots go to the lowest indices)

@@ -63,3 +63,43 @@ def plan(counts, resident, costs: dict, n_stage: int) -> list[int]:
     for _, e in savings[:n_stage]:
         where[e] = STAGED
     return where
+
+
+def plan_balanced(counts, resident, costs: dict, n_stage: int) -> list[int]:
+    """The balanced plan (an extension beyond the page, same latency model):
+    the host and the host-to-GPU link work in parallel, so a batch's
+    non-resident experts cost max(host time, link time), with host time the
+    sum of cpu(n) of the experts left on the host and link time the sum of
+    gpu(n) of the staged ones.  Candidates (active, not resident) are ranked
+    by cpu(n) / gpu(n), largest first (gpu(n) <= 0 ranks first; equal ratios:
+    lower index first); the plan stages the first j of them, j in
+    0..min(n_stage, #candidates) minimising that maximum (equal maxima: the
+    smaller j).  Sums run in rank order."""
+    where = []
+    cand = []
+    for e, n in enumerate(counts):
+        n = int(n)
+        if n == 0:
+            where.append(IDLE)
+        elif resident[e]:
+            where.append(RESIDENT)
+        else:
+            where.append(CPU)
+            c, g = cpu_latency(costs, n), gpu_latency(costs, n)
+            ratio = float("inf") if g <= 0 else c / g
+            cand.append((ratio, e, c, g))
+    cand.sort(key=lambda item: (-item[0], item[1]))
+    best_j, best = 0, None
+    for j in range(min(n_stage, len(cand)) + 1):
+        host = 0.0
+        for i in range(j, len(cand)):
+            host += cand[i][2]
+        link = 0.0
+        for i in range(j):
+            link += cand[i][3]
+        cost = max(host, link)
+        if best is None or cost < best:
+            best_j, best = j, cost
+    for i in range(best_j):
+        where[cand[i][1]] = STAGED
+    return where

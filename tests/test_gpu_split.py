@@ -31,6 +31,8 @@ def expected_plan(ids, E, resident, policy, costs, n_stage, moe):
         c = dict(cpu_us=0.0, cpu_us_per_token=0.0, xfer_us=BIG, gpu_us=0.0, gpu_us_per_token=0.0)
     elif policy == moe.POLICY_ALL_STAGED:
         c = dict(cpu_us=BIG, cpu_us_per_token=0.0, xfer_us=0.0, gpu_us=0.0, gpu_us_per_token=0.0)
+    elif policy == moe.POLICY_BALANCED:
+        return osplit.plan_balanced(counts, resident, costs, n_stage)
     else:
         c = costs
     return osplit.plan(counts, resident, c, n_stage)
@@ -70,6 +72,15 @@ def test_single_token(policy):
 def test_dynamic_mix(T):
     # more experts would gain from a copy than there are slots: some go to the host
     run_case(T, 8, 2, 256, 512, [0, 1, 0, 0, 1, 0, 0, 1], 2, 0, COSTS, seed=T, skew=1.0)
+
+
+@pytest.mark.parametrize("T", [40, 300])
+def test_balanced_mix(T):
+    # host and link both busy: the balanced plan stages a prefix of the ranked experts
+    costs = dict(cpu_us=50.0, cpu_us_per_token=1.0, xfer_us=150.0, gpu_us=0.0,
+                 gpu_us_per_token=0.0)
+    layer = run_case(T, 8, 2, 256, 512, [0, 1, 0, 0, 0, 0, 0, 1], 3, 3, costs, seed=T + 1)
+    assert 0 < list(layer.where).count(3) and 0 < list(layer.where).count(2)
 
 
 def test_everything_on_host():

@@ -100,3 +100,73 @@ def test_plan_staged_set_by_brute_force(seed):
             assert where[e] == osplit.RESIDENT
         else:
             assert where[e] == (osplit.STAGED if e in staged else osplit.CPU), (e, where)
+
+
+def makespan(where, counts, costs):
+    host = sum(osplit.cpu_latency(costs, counts[e]) for e in range(len(counts))
+               if where[e] == osplit.CPU)
+    link = sum(osplit.gpu_latency(costs, counts[e]) for e in range(len(counts))
+               if where[e] == osplit.STAGED)
+    return max(host, link)
+
+
+def test_balanced_hand_case():
+    # four experts of 128 tokens: host 5.0 ms each, copy 6.4 ms each;
+    # staging two gives max(10.0, 12.8) = 12.8 ms, the best prefix
+    costs = dict(cpu_us=1700.0, cpu_us_per_token=25.78125, xfer_us=6400.0, gpu_us=0.0,
+                 gpu_us_per_token=0.0)
+    counts = [128, 0, 128, 128, 128]
+    resident = [0, 1, 0, 0, 0]
+    where = osplit.plan_balanced(counts, resident, costs, n_stage=4)
+    assert where == [osplit.STAGED, osplit.IDLE, osplit.STAGED, osplit.CPU, osplit.CPU]
+    assert makespan(where, counts, costs) == 12800.0
+    # the per-expert rule keeps all four on the host (5.0 < 6.4): 20 ms
+    assert osplit.plan(counts, resident, costs, 4) == [osplit.CPU, osplit.IDLE, osplit.CPU,
+                                                       osplit.CPU, osplit.CPU]
+    # with one slot: max(15.0, 6.4)
+    assert osplit.plan_balanced(counts, resident, costs, 1).count(osplit.STAGED) == 1
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_balanced_with_equal_experts_is_optimal(seed):
+    """When every candidate has the same token count the ranking is only the
+    index order and the best prefix is the best subset: checked against all
+    subsets; and in general the plan is never worse than staging nothing."""
+    rng = random.Random(2000 + seed)
+    E = rng.randint(1, 9)
+    n = rng.choice([1, 16, 128, 512])
+    counts = [n if rng.random() < 0.8 else 0 for _ in range(E)]
+    resident = [rng.random() < 0.25 for _ in range(E)]
+    costs = dict(cpu_us=rng.uniform(0, 3000), cpu_us_per_token=rng.uniform(0, 60),
+                 xfer_us=rng.uniform(100, 8000), gpu_us=0.0, gpu_us_per_token=0.0)
+    n_stage = rng.randint(0, E)
+    where = osplit.plan_balanced(counts, resident, costs, n_stage)
+    cand = [e for e in range(E) if counts[e] and not resident[e]]
+    best = min(makespan([osplit.STAGED if e in set(sub) else
+                         (osplit.CPU if e in cand else osplit.IDLE) for e in range(E)],
+                        counts, costs)
+               for m in range(min(n_stage, len(cand)) + 1)
+               for sub in itertools.combinations(cand, m))
+    assert makespan(where, counts, costs) == pytest.approx(best, rel=1e-12)
+    for e in range(E):
+        if counts[e] == 0:
+            assert where[e] == osplit.IDLE
+        elif resident[e]:
+            assert where[e] == osplit.RESIDENT
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_balanced_never_worse_than_fixed_plans(seed):
+    rng = random.Random(3000 + seed)
+    E = rng.randint(1, 12)
+    counts = [rng.choice([0, 1, 3, 16, 64, 128, 300, 700]) for _ in range(E)]
+    resident = [rng.random() < 0.3 for _ in range(E)]
+    costs = dict(cpu_us=rng.uniform(0, 3000), cpu_us_per_token=rng.uniform(0, 60),
+                 xfer_us=rng.uniform(100, 8000), gpu_us=rng.uniform(0, 100),
+                 gpu_us_per_token=rng.uniform(0, 1))
+    n_stage = rng.randint(0, E)
+    where = osplit.plan_balanced(counts, resident, costs, n_stage)
+    assert where.count(osplit.STAGED) <= n_stage
+    cand = [e for e in range(E) if counts[e] and not resident[e]]
+    all_cpu = [osplit.CPU if e in cand else where[e] for e in range(E)]
+    assert makespan(where, counts, costs) <= makespan(all_cpu, counts, costs)

@@ -44,6 +44,22 @@ def test_plan_matches_oracle(L, seed):
     assert list(got) == osplit.plan(counts, resident, costs, n_stage)
 
 
+@pytest.mark.parametrize("seed", range(25))
+def test_balanced_plan_matches_oracle(L, seed):
+    rng = random.Random(500 + seed)
+    E = rng.randint(1, 256)
+    counts = [rng.choice([0, 0, 1, 2, 16, 64, 128, 128, 500]) for _ in range(E)]
+    resident = [int(rng.random() < 0.4) for _ in range(E)]
+    costs = dict(cpu_us=rng.uniform(0, 3000), cpu_us_per_token=rng.uniform(0, 60),
+                 xfer_us=rng.uniform(0, 8000), gpu_us=rng.uniform(0, 50),
+                 gpu_us_per_token=rng.uniform(0, 1))
+    if seed % 5 == 0:
+        costs.update(xfer_us=0.0, gpu_us=0.0, gpu_us_per_token=0.0)   # gpu(n) = 0: ranks first
+    n_stage = rng.randint(0, 16)
+    got = L.split_plan(counts, resident, L.split_costs(**costs), n_stage, balanced=True)
+    assert list(got) == osplit.plan_balanced(counts, resident, costs, n_stage)
+
+
 def test_plan_and_place_errors(L):
     lib = L.lib()
     c = L.split_costs()
@@ -89,16 +105,17 @@ def test_host_layout(L):
 
 @pytest.mark.parametrize("H,I,n", [(64, 64, 1), (128, 256, 3), (256, 192, 8), (192, 320, 13),
                                    (512, 128, 33)])
-@pytest.mark.parametrize("portable", [False, True])
-def test_host_expert_matches_oracle(L, H, I, n, portable):
-    if not portable and L.host_isa() != L.HOST_ISA_AVX512_BF16:
+@pytest.mark.parametrize("path", ["auto", "avx512_bf16", "portable"])
+def test_host_expert_matches_oracle(L, H, I, n, path):
+    need = {"auto": 0, "avx512_bf16": L.HOST_ISA_AVX512_BF16, "portable": 0}[path]
+    if L.host_isa() < need:
         pytest.skip("this CPU has no AVX512_BF16")
     Wg, Wu, Wd = master(1, H, I, seed=H + I + n)
     g = torch.Generator().manual_seed(n)
     x = torch.randn(n, H, generator=g).to(torch.bfloat16)
     w = torch.rand(n, generator=g) + 0.25
     packed = L.host_pack_weights(Wg, Wu, Wd)
-    h, y = L.host_expert_ffn(packed[0], x, w, portable=portable)
+    h, y = L.host_expert_ffn(packed[0], x, w, path=path)
     ids = np.zeros((n, 1), np.int32)
     ref = oracle.moe_layer(x, ids, w.double().numpy()[:, None], Wg, Wu, Wd)
     err = rel_err(y.double().numpy(), ref)
@@ -111,18 +128,20 @@ def test_host_expert_matches_oracle(L, H, I, n, portable):
     assert rel_err(h.double().numpy(), hd.numpy()) <= 1e-2
 
 
-def test_host_paths_agree(L):
-    if L.host_isa() != L.HOST_ISA_AVX512_BF16:
-        pytest.skip("this CPU has no AVX512_BF16")
-    H, I, n = 256, 512, 9
+@pytest.mark.parametrize("n", [9, 16, 40])
+def test_host_paths_agree(L, n):
+    """Every instruction-set path this CPU has against the portable one: fp32
+    sums in a different order, so a few bf16 ulps at most."""
+    H, I = 256, 512
     Wg, Wu, Wd = master(1, H, I, seed=5)
     x = torch.randn(n, H, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
     w = torch.ones(n)
     packed = L.host_pack_weights(Wg, Wu, Wd)
-    _, y0 = L.host_expert_ffn(packed[0], x, w, portable=False)
-    _, y1 = L.host_expert_ffn(packed[0], x, w, portable=True)
-    # fp32 sums in a different order: a few bf16 ulps at most
-    assert rel_err(y0.double().numpy(), y1.double().numpy()) <= 4e-3
+    _, y1 = L.host_expert_ffn(packed[0], x, w, path="portable")
+    paths = ["auto"] + (["avx512_bf16"] if L.host_isa() >= L.HOST_ISA_AVX512_BF16 else [])
+    for p in paths:
+        _, y0 = L.host_expert_ffn(packed[0], x, w, path=p)
+        assert rel_err(y0.double().numpy(), y1.double().numpy()) <= 4e-3, p
 
 
 def test_host_threads_do_not_change_result(L):
