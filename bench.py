@@ -804,6 +804,10 @@ class SplitBench:
                            for b in range(NBATCH)] for T in self.Ts}
         self.outs = {T: torch.empty((T, self.H), dtype=torch.bfloat16, device=dev)
                      for T in self.Ts}
+        # tokens per expert of each batch (for the launch count of a call)
+        self.counts = {T: [torch.bincount(moe.route_topk(lg, self.k)[0].flatten().long(),
+                                          minlength=self.E).cpu().tolist()
+                           for _, lg in self.dev_in[T]] for T in self.Ts}
 
     def measure(self, clk):
         args, layer = self.args, self.layer
@@ -819,6 +823,7 @@ class SplitBench:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 places = {"resident": 0, "staged": 0, "cpu": 0}
+                launches = 0
                 e0.record()
                 for i in range(args.steps):
                     x, lg = self.dev_in[T][i % NBATCH]
@@ -827,16 +832,33 @@ class SplitBench:
                     places["resident"] += w.count(self.moe.SPLIT_RESIDENT)
                     places["staged"] += w.count(self.moe.SPLIT_STAGED)
                     places["cpu"] += w.count(self.moe.SPLIT_CPU)
+                    launches += self.kernels_per_call(T, w, self.counts[T][i % NBATCH])
                 e1.record()
                 torch.cuda.synchronize()
                 if layer.check() != 0:
                     raise RuntimeError("split: device status word reports a fault")
                 ms = e0.elapsed_time(e1) / args.steps
                 mean = {key: v / args.steps for key, v in places.items()}
-                res[(T, pname)] = dict(ms=ms, places=mean,
+                res[(T, pname)] = dict(ms=ms, places=mean, launches=launches,
                                        bytes={key: v * expert_bytes for key, v in mean.items()})
         clk.mark_end()
         return res
+
+    def kernels_per_call(self, T, where, counts):
+        """Kernels one moe_split_forward launches: route, slot map, the
+        permutation (one kernel up to 2048 assignments, else three), per GPU
+        group of experts (resident, staged) a gate/up and a down GEMM plus a
+        gather kernel for CTA-pair tiles, and the combine."""
+        A = T * self.k
+        n = 2 + (1 if A <= CHUNK else 3) + 1
+        for kind in (self.moe.SPLIT_RESIDENT, self.moe.SPLIT_STAGED):
+            ex = [e for e in range(self.E) if where[e] == kind]
+            if not ex:
+                continue
+            n += 2
+            if gemm_token_cap(sum(counts[e] for e in ex), 1, len(ex)) > 64:
+                n += 1
+        return n
 
     def report(self, res, clocks):
         hbm, _, src = peaks()
@@ -895,8 +917,10 @@ class SplitBench:
                              "note": "ideal = max(host experts' bytes / host read bandwidth, "
                                      "staged bytes / link + GPU experts' bytes / HBM)"},
                 "per_T": per_T, "clocks": clocks,
-                "gpu_launches_per_call": "route, slot map, permute, gate/up + down per GPU "
-                                         "group, combine"}
+                "gpu_launches": sum(res[(T, "dynamic")]["launches"] for T in self.Ts),
+                "gpu_launches_note": "timed calls of the dynamic policy: route, slot map, "
+                                     "permutation, gate/up and down GEMMs (+ gather for pair "
+                                     "tiles) per GPU group of experts, combine"}
 
     def host_kernel_rates(self, ns=(1, 16, 64, 128, 512)):
         """moe_host_expert_ffn alone on expert 0 (all host threads, the best of
