@@ -196,6 +196,9 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
  *   host_ws            host workspace (page-locked), moe_split_host_workspace_size
  *                      bytes; it must stay untouched until the stream has
  *                      finished the call
+ * Calls that share staging slots or workspaces must be ordered: issue them
+ * on one stream (each call's synchronisation then covers the previous one's
+ * use of the slots).
  * Exceptions to moe.h's conventions: this call synchronises `stream` once
  * (after step 1: the plan needs the batch's routing) and computes on the
  * calling thread and the host pool; it returns once steps 3-5 are enqueued.

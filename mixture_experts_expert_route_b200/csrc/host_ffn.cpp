@@ -104,9 +104,18 @@ class HostPool {
 };
 
 HostPool& pool() {
-    // created on first use and never destroyed: its threads wait on a
-    // condition variable until the process exits
-    static HostPool* p = new HostPool(static_cast<int>(std::thread::hardware_concurrency()));
+    // Created on first use and never destroyed: its threads wait on a
+    // condition variable until the process exits.  A child process made by
+    // fork() has none of its parent's threads, so it gets a pool of its own
+    // (the parent's object is left alone).
+    static std::mutex mu;
+    static HostPool* p = nullptr;
+    static pid_t owner = 0;
+    std::lock_guard<std::mutex> g(mu);
+    if (!p || owner != getpid()) {
+        p = new HostPool(static_cast<int>(std::thread::hardware_concurrency()));
+        owner = getpid();
+    }
     return *p;
 }
 

@@ -189,3 +189,38 @@ def test_split_forward_argument_errors(L):
     a.T = 4
     a.n_stage = 254                                                             # 1 + 2 + 254
     assert lib.moe_split_forward(ctypes.byref(a), None, 0, None, 0, None) == 2
+
+
+def test_host_kernel_in_a_forked_child(L):
+    """A child made by fork() after the parent used the host kernel gets its
+    own thread pool (the parent's threads do not exist in it)."""
+    import os
+    import signal
+    import time
+    import warnings
+    H, I = 64, 128
+    Wg, Wu, Wd = master(1, H, I, seed=2)
+    packed = L.host_pack_weights(Wg, Wu, Wd)
+    x = torch.randn(5, H, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    w = torch.ones(5)
+    _, y0 = L.host_expert_ffn(packed[0], x, w)
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore", DeprecationWarning)
+        pid = os.fork()
+    if pid == 0:
+        try:
+            _, y1 = L.host_expert_ffn(packed[0], x, w)
+            os._exit(0 if torch.equal(y0, y1) else 3)
+        except BaseException:
+            os._exit(4)
+    deadline = time.time() + 60
+    while True:
+        done, status = os.waitpid(pid, os.WNOHANG)
+        if done:
+            break
+        if time.time() > deadline:
+            os.kill(pid, signal.SIGKILL)
+            os.waitpid(pid, 0)
+            pytest.fail("the forked child did not finish")
+        time.sleep(0.05)
+    assert os.WIFEXITED(status) and os.WEXITSTATUS(status) == 0
