@@ -31,7 +31,8 @@
  *   - Process-wide state is limited to two things: the per-device opt-in of
  *     the GEMM kernels to more than 48 KB of shared memory (set on the first
  *     launch on each device, read-only afterwards), and the fixed scratch
- *     array of moe_align_permute_noalloc (see its entry).  Apart from
+ *     array of moe_align_permute_noalloc (see its entry).  The CPU/GPU split
+ *     of moe_split.h adds its host thread pool (see there).  Apart from
  *     moe_align_permute_noalloc, calls on different streams with separate
  *     buffers may run concurrently.
  */

@@ -20,6 +20,12 @@
  * the host's rows join the combine.  bf16 only.  The conventions of moe.h
  * apply, with the exceptions stated at moe_split_forward (it synchronises its
  * stream once and reads and writes host memory).
+ *
+ * Process-wide state: the host functions share one thread pool (one thread
+ * per hardware thread, created on first use, one pool per process: a child
+ * made by fork() builds its own; calls from several threads take turns), and
+ * the first host call asks Linux once for the AMX tile state where the CPU
+ * has AMX.
  */
 #ifndef MOE_B200_SPLIT_H
 #define MOE_B200_SPLIT_H

@@ -10,6 +10,8 @@
 // batch's token count.  The slot permutation keeps every GPU expert's rows
 // where the layer's grouped GEMMs and combine expect them, and puts the host
 // experts' rows first (slot 0), in the order the host produces them.
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <chrono>
 #include <cstring>
@@ -144,6 +146,14 @@ int group_nmax(const std::vector<int>& counts, const int32_t* where, int E, int 
     return n ? gemm_nmax_for(static_cast<int>(A), 1, n) : 0;
 }
 
+// NVTX range over one step of the split (free when no profiler is attached)
+struct Range {
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range&) = delete;
+    Range& operator=(const Range&) = delete;
+};
+
 double now_us() {
     return std::chrono::duration<double, std::micro>(
                std::chrono::steady_clock::now().time_since_epoch())
@@ -255,17 +265,23 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     const int cap = moe_permute_capacity(T, k, Es, block_m);
     int32_t* status = a->status ? a->status : d.ctl;
 
+    Range whole("moe_split_forward");
     // 1. route on the GPU, bring the routing and x to the host
-    if (!a->status && cudaMemsetAsync(d.ctl, 0, 64 * sizeof(int32_t), s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    if (launch_route_topk(a->logits, T, E, k, d.ids, d.w, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaMemcpyAsync(hb.ids, d.ids, sizeof(int32_t) * A, cudaMemcpyDeviceToHost, s) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(hb.w, d.w, sizeof(float) * A, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(hb.x, a->x, sizeof(uint16_t) * T * static_cast<size_t>(H),
-                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    {
+        Range r("moe split: route, routing to the host");
+        if (!a->status && cudaMemsetAsync(d.ctl, 0, 64 * sizeof(int32_t), s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (launch_route_topk(a->logits, T, E, k, d.ids, d.w, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaMemcpyAsync(hb.ids, d.ids, sizeof(int32_t) * A, cudaMemcpyDeviceToHost, s) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(hb.w, d.w, sizeof(float) * A, cudaMemcpyDeviceToHost, s) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(hb.x, a->x, sizeof(uint16_t) * T * static_cast<size_t>(H),
+                            cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
 
     // 2. the plan
     std::vector<int> counts(E, 0);
@@ -293,6 +309,7 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     if (a->where) std::memcpy(a->where, where.data(), sizeof(int32_t) * E);
 
     // 3. slots, weight copies, slot permutation, the GPU experts
+    Range gpu_part("moe split: weight copies, slot permutation, GPU experts");
     std::vector<int> staged;
     {
         int r = 0;
@@ -356,6 +373,7 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
 
     // 4. the host experts, while the GPU runs; their rows go to slot 0 in
     // ascending flat index, the order the stable permutation gives them
+    Range host_part("moe split: host experts, combine");
     std::vector<int> pos(A, -1);
     int n_cpu = 0;
     for (long f = 0; f < A; ++f)
