@@ -157,8 +157,10 @@ def kernels_per_forward(T, k, E, fp8, H, lora=False):
     small = T <= SMALL_T and A <= CHUNK
     if small:
         n = 1                                   # fused route + permute
+    elif A <= CHUNK:
+        n = 2                                   # route, single-CTA permute
     else:
-        n = 1 + (1 if A <= CHUNK else 3)        # route, permute (1 or 3 kernels)
+        n = 3                                   # route, count, scan + scatter
     # FP8: amax(x) and the codes of x (in the route kernel for small batches)
     n += 2 if fp8 and not (small and T * H <= SMALL_AMAX) else 0
     # gather (pair tiles and adapter layers; else in the GEMM), adapter shrinks
@@ -850,7 +852,7 @@ class SplitBench:
         group of experts (resident, staged) a gate/up and a down GEMM plus a
         gather kernel for CTA-pair tiles, and the combine."""
         A = T * self.k
-        n = 2 + (1 if A <= CHUNK else 3) + 1
+        n = 2 + (1 if A <= CHUNK else 2) + 1
         for kind in (self.moe.SPLIT_RESIDENT, self.moe.SPLIT_STAGED):
             ex = [e for e in range(self.E) if where[e] == kind]
             if not ex:

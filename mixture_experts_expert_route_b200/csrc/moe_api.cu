@@ -577,7 +577,6 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     // kernels are done with it.
     cudaError_t e;
     const long x_elems = static_cast<long>(a->T) * a->H;
-    const long A = static_cast<long>(a->T) * a->k;
     const bool fp8 = a->dtype == MOE_FP8_E4M3;
     const bool small = fused_route_permute_ok(a->T, a->k);
     // FP8 with a small x: the single-CTA route kernel also takes amax(x) and
@@ -605,9 +604,10 @@ moe_status moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, moe
     FfnCall f{a->dtype, a->T, a->k, a->E, a->H, a->I, cap, a->x, w, b.counts, b.offsets,
               b.sorted_ids, a->packed, a->scales, b.y_out, status, a->max_ctas};
     f.x_ready = x_fused;
-    // the single-CTA permutation (the only one for A <= 2048) is the kernel
-    // right before the gate/up GEMM, unless FP8 kernels come between
-    f.counts_from_prev = permute_chunks(A) <= 1;
+    // the permutation's last kernel (the single-CTA one, or scan + scatter,
+    // which writes the counts) runs right before the gate/up GEMM, unless
+    // FP8 or gather kernels come between (run_ffn clears the flag then)
+    f.counts_from_prev = true;
     f.combine = pick_combine(a->combine);
     f.lora = a->lora;
     st = run_ffn(f, b.ffn, ev, s);

@@ -342,51 +342,55 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Scan + scatter: every CTA sums the per-chunk counts itself (all chunks for
+// the expert totals and padded offsets, the chunks before its own for its
+// start positions), so no separate scan kernel runs; CTA 0 also writes the
+// counts, offsets, tile list and pads.  Then the chunk's assignments are
+// placed as in the single-CTA kernel.
 __global__ void __launch_bounds__(kThreads)
-    permute_scan_kernel(int nchunks, int E, int block_m, int capacity, int32_t* chunk_counts,
-                        int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* tiles,
-                        int32_t* num_tiles) {
+    scan_scatter_kernel(const int32_t* ids, long A, int E, int block_m, int capacity,
+                        int nchunks, const int32_t* __restrict__ chunk_counts, int32_t* counts,
+                        int32_t* offsets, int32_t* sorted_ids, int32_t* __restrict__ inv_perm,
+                        int32_t* tiles, int32_t* num_tiles) {
     constexpr int NW = kThreads / 32;
+    __shared__ int hist[NW][kMaxExperts];
     __shared__ int tmp[NW + 1];
     pdl_wait();
     pdl_trigger();
     const int e = threadIdx.x;
-    int run = 0;
+    const int me = blockIdx.x;
+    int total = 0, before = 0;
     if (e < E)
         for (int c0 = 0; c0 < nchunks; c0 += kScanBatch) {
-            // the batch's loads are independent: issue them all, then scan
+            // the batch's loads are independent: issue them all, then add
             int v[kScanBatch];
 #pragma unroll
             for (int i = 0; i < kScanBatch; ++i)
                 v[i] = c0 + i < nchunks ? chunk_counts[static_cast<long>(c0 + i) * E + e] : 0;
 #pragma unroll
             for (int i = 0; i < kScanBatch; ++i) {
-                if (c0 + i < nchunks) chunk_counts[static_cast<long>(c0 + i) * E + e] = run;
-                run += v[i];
+                if (c0 + i < me) before += v[i];
+                total += v[i];
             }
         }
-    finish_offsets<kThreads>(run, E, block_m, counts, offsets, sorted_ids, tiles, num_tiles, tmp);
-    const int total = tmp[NW];
-    __syncthreads();
-    fill_tail<kThreads>(total, block_m, capacity, sorted_ids, tiles);
-}
-
-__global__ void __launch_bounds__(kThreads)
-    permute_scatter_kernel(const int32_t* ids, long A, int E,
-                           const int32_t* __restrict__ chunk_prefix,
-                           const int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
-                           int32_t* __restrict__ inv_perm) {
-    constexpr int NW = kThreads / 32;
-    __shared__ int hist[NW][kMaxExperts];
-    pdl_wait();
-    pdl_trigger();
+    int o;
+    if (me == 0) {
+        o = finish_offsets<kThreads>(total, E, block_m, counts, offsets, sorted_ids, tiles,
+                                     num_tiles, tmp);
+        const int all = tmp[NW];
+        __syncthreads();
+        fill_tail<kThreads>(all, block_m, capacity, sorted_ids, tiles);
+    } else {
+        const int padded = e < E ? (total + block_m - 1) / block_m * block_m : 0;
+        o = block_exclusive_scan<kThreads>(padded, tmp);
+    }
     for (int i = threadIdx.x; i < NW * kMaxExperts; i += kThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    const long base = static_cast<long>(blockIdx.x) * kPermChunk;
+    const long base = static_cast<long>(me) * kPermChunk;
     chunk_histogram<NW, kPermChunk>(ids, A, base, E, hist, nullptr);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-        int run = offsets[e] + chunk_prefix[static_cast<long>(blockIdx.x) * E + e];
+    if (e < E) {
+        int run = o + before;
         for (int wq = 0; wq < NW; ++wq) {
             const int h = hist[wq][e];
             hist[wq][e] = run;
@@ -398,6 +402,15 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 int epl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
+
+cudaError_t launch_scan_scatter(const int32_t* ids, long A, int E, int block_m, int capacity,
+                                int nch, const int32_t* chunk_counts, int32_t* counts,
+                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
+                                int32_t* tiles, int32_t* num_tiles, cudaStream_t s) {
+    return launch_pdl(scan_scatter_kernel, dim3(nch), dim3(kThreads), 0, s, ids, A, E, block_m,
+                      capacity, nch, chunk_counts, counts, offsets, sorted_ids, inv_perm, tiles,
+                      num_tiles);
+}
 
 }  // namespace
 
@@ -460,12 +473,8 @@ cudaError_t launch_align_permute(const int32_t* ids, int T, int k, int E, int bl
     cudaError_t e = launch_pdl(permute_count_kernel, dim3(nch), dim3(kThreads), 0, s, ids, A, E,
                                chunk_counts, status);
     if (e == cudaSuccess)
-        e = launch_pdl(permute_scan_kernel, dim3(1), dim3(kThreads), 0, s, nch, E, block_m,
-                       capacity, chunk_counts, counts, offsets, sorted_ids, tiles, num_tiles);
-    if (e == cudaSuccess)
-        e = launch_pdl(permute_scatter_kernel, dim3(nch), dim3(kThreads), 0, s, ids, A, E,
-                       static_cast<const int32_t*>(chunk_counts),
-                       static_cast<const int32_t*>(offsets), sorted_ids, inv_perm);
+        e = launch_scan_scatter(ids, A, E, block_m, capacity, nch, chunk_counts, counts, offsets,
+                                sorted_ids, inv_perm, tiles, num_tiles, s);
     return e;
 }
 

@@ -76,13 +76,15 @@ def test_bench_mirrors_library_dispatch_constants():
     assert bench.kernels_per_forward(1, 2, 8, False, 4096) == 4
     # FP8 T=1, x of 5.6 KB: amax and x codes in the route kernel, plus h quantisation
     assert bench.kernels_per_forward(1, 4, 32, True, 2880) == 5
-    # FP8 T=2048: route, 3 permutation kernels, amax, x codes, gather, 2 GEMMs,
-    # quant, finalize
-    assert bench.kernels_per_forward(2048, 4, 32, True, 2880) == 11
-    # prefill bf16 T=4096: route, 3 permutation kernels, gather, 2 GEMMs, finalize
-    assert bench.kernels_per_forward(4096, 8, 128, False, 2048) == 8
+    # FP8 T=2048: route, count, scan + scatter, amax, x codes, gather, 2 GEMMs,
+    # quant, combine
+    assert bench.kernels_per_forward(2048, 4, 32, True, 2880) == 10
+    # prefill bf16 T=4096: route, count, scan + scatter, gather, 2 GEMMs, combine
+    assert bench.kernels_per_forward(4096, 8, 128, False, 2048) == 7
+    # token cap 64 (no gather kernel): route, count, scan + scatter, 2 GEMMs, combine
+    assert bench.kernels_per_forward(1000, 3, 96, False, 128) == 6
     # with adapters: the gather kernel and two shrink GEMMs more
-    assert bench.kernels_per_forward(4096, 8, 128, False, 2048, lora=True) == 10
+    assert bench.kernels_per_forward(4096, 8, 128, False, 2048, lora=True) == 9
     assert bench.kernels_per_forward(1, 2, 8, False, 4096, lora=True) == 7
     # the token-tile cap (pair tiles above 64): twice the mean per expert
     assert bench.gemm_token_cap(64, 2, 8) == 32

@@ -139,6 +139,12 @@ LAYER_CASES = [
     ("tiny", 9, 1, 1, 256, 256),         # E = 1: dense SwiGLU
     ("tiny", 40, 2, 2, 256, 256),        # pair tiles, token cap 2*mean = 80 (not a multiple of 32)
     ("tiny", 56, 2, 2, 192, 128),        # pair tiles, 2*mean = 112
+    # past the single-CTA permutation (T*k > 2048): route, count, scan+scatter
+    ("tiny", 1100, 8, 2, 256, 256),      # 5 chunks, pair tiles (gather kernel between)
+    ("tiny", 300, 128, 8, 128, 128),     # 5 chunks, one-CTA tiles: the GEMM follows scan+scatter
+    ("tiny", 520, 64, 8, 128, 192),      # 9 chunks, pair tiles
+    ("tiny", 800, 16, 3, 128, 192),      # k = 3, pair tiles
+    ("tiny", 1000, 96, 3, 128, 128),     # k = 3, one-CTA tiles
 ]
 
 
