@@ -646,7 +646,10 @@ class Bench:
                 # own adapter on the three matrices (2r(H+I) MACs each)
                 n_ad = int((self.adapters[T] >= 0).sum().item())
                 layer_flops += 6.0 * n_ad * k * 2 * self.lora_rank * (H + I)
-            lt = r["layer_graph_ms"].get(T, r["layer_direct_ms"][T])
+            # one token count: the primary timed region is that T's layer time (the
+            # per-T region repeats it later, on a warmer, power-capped GPU)
+            lt = (r["elapsed_ms"] / self.args.steps if len(Ts) == 1
+                  else r["layer_graph_ms"].get(T, r["layer_direct_ms"][T]))
             per_T[str(T)] = {
                 "layer_us": round(1e3 * lt, 2),
                 "layer_us_direct": round(1e3 * r["layer_direct_ms"][T], 2),
