@@ -829,10 +829,18 @@ class SplitBench:
                 e1 = torch.cuda.Event(enable_timing=True)
                 places = {"resident": 0, "staged": 0, "cpu": 0}
                 launches = 0
+                # each call is bracketed by its own events (a call waits for the
+                # routing once, so back-to-back calls do not overlap anyway); the
+                # median of the calls is reported beside the mean, because the
+                # host's cores are shared with other work on the machine
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(args.steps)]
                 e0.record()
                 for i in range(args.steps):
                     x, lg = self.dev_in[T][i % NBATCH]
+                    evs[i][0].record()
                     layer(x, lg, out=self.outs[T], policy=pol)
+                    evs[i][1].record()
                     w = list(layer.where)
                     places["resident"] += w.count(self.moe.SPLIT_RESIDENT)
                     places["staged"] += w.count(self.moe.SPLIT_STAGED)
@@ -842,9 +850,11 @@ class SplitBench:
                 torch.cuda.synchronize()
                 if layer.check() != 0:
                     raise RuntimeError("split: device status word reports a fault")
-                ms = e0.elapsed_time(e1) / args.steps
+                per_call = [a.elapsed_time(b) for a, b in evs]
+                ms = statistics.median(per_call)
                 mean = {key: v / args.steps for key, v in places.items()}
-                res[(T, pname)] = dict(ms=ms, places=mean, launches=launches,
+                res[(T, pname)] = dict(ms=ms, mean_ms=e0.elapsed_time(e1) / args.steps,
+                                       places=mean, launches=launches,
                                        bytes={key: v * expert_bytes for key, v in mean.items()})
         clk.mark_end()
         return res
@@ -881,6 +891,7 @@ class SplitBench:
                            b["staged"] / (link * 1e9) + (b["resident"] + b["staged"]) /
                            (hbm * 1e9)) * 1e3
             entry = {"layer_us": round(1e3 * d["ms"], 1),
+                     "layer_us_mean": round(1e3 * d["mean_ms"], 1),
                      "tokens_per_s": round(T / (d["ms"] / 1e3), 1),
                      "experts_per_call": {k2: round(v, 2) for k2, v in d["places"].items()},
                      "ideal_us": round(1e3 * ideal_ms, 1),
@@ -906,7 +917,7 @@ class SplitBench:
                 "value": round(sum(self.Ts) / (total_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(total_ms, 3), "dtype": "bf16",
                 "policy": "dynamic (the per-expert rule); balanced_* fields: the host/link "
-                          "balanced plan",
+                          "balanced plan; *_us: median over the timed calls",
                 "value_balanced": round(sum(self.Ts) / (total_bal / 1e3), 1),
                 "resident": [int(v) for v in self.resident],
                 "costs": {"cpu_us": round(c.cpu_us, 1),

@@ -187,9 +187,11 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
  *                      experts in ascending index (E = S); NULL when S = 0
  *   stage_packed       device, moe_pack_weights layout with n_stage experts
  *                      (overwritten by the copies); NULL when n_stage = 0
- *   host_packed        host (page-locked for asynchronous copies),
- *                      moe_pack_weights layout of all E experts: the source
- *                      of the copies
+ *   host_packed        host (page-locked for asynchronous copies): for each
+ *                      expert e in turn, the moe_pack_weights output of that
+ *                      expert alone (E = 1, moe_packed_weights_size(MOE_BF16,
+ *                      1, H, I) bytes each): the source of the copies, so that
+ *                      set-up can pack one expert at a time
  *   host_weights       host, moe_host_pack_weights layout of all E experts
  *   costs              latency model (DYNAMIC, BALANCED); may be NULL otherwise
  *   where              optional host int32 [E] out: the plan that ran

@@ -467,11 +467,15 @@ class SplitLayer:
         self.S = int(self.resident.sum())
         E, H, I = self.E, self.H, self.I
         self.host_weights = host_pack_weights(Wg, Wu, Wd)
-        # the GPU layout of all experts, made on the device once and kept in
-        # page-locked host memory as the source of the staging copies
-        pk, _ = pack_weights(BF16, Wg.to(self.device), Wu.to(self.device), Wd.to(self.device))
-        self.host_packed = torch.empty(pk.numel(), dtype=torch.uint8, pin_memory=True)
-        self.host_packed.copy_(pk)
+        # the GPU layout of each expert, made on the device one expert at a
+        # time and kept in page-locked host memory as the source of the
+        # staging copies (the GPU never holds more than one expert's copy)
+        per = lib().moe_packed_weights_size(BF16, 1, H, I)
+        self.host_packed = torch.empty((E, per), dtype=torch.uint8, pin_memory=True)
+        for e in range(E):
+            pk, _ = pack_weights(BF16, Wg[e:e + 1].to(self.device), Wu[e:e + 1].to(self.device),
+                                 Wd[e:e + 1].to(self.device))
+            self.host_packed[e].copy_(pk)
         del pk
         idx = [e for e in range(E) if self.resident[e]]
         self.resident_packed = None

@@ -328,19 +328,20 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
         cudaSuccess)
         return MOE_ERR_CUDA;
     if (!staged.empty()) {
-        const PackedGeom all = packed_geom(0, E, H, I);
+        // host_packed: expert e's own packed layout (E = 1) at e * (gate/up +
+        // down bytes); the staging buffer: the packed layout of n_stage experts
         const PackedGeom one = packed_geom(0, 1, H, I);
         const PackedGeom stg = packed_geom(0, a->n_stage, H, I);
+        const size_t per_expert = one.gu_bytes + one.dn_bytes;
         cudaStream_t cs = a->copy_stream ? reinterpret_cast<cudaStream_t>(a->copy_stream) : s;
         const char* src = static_cast<const char*>(a->host_packed);
         char* dst = static_cast<char*>(a->stage_packed);
         for (size_t j = 0; j < staged.size(); ++j) {
-            const size_t e = static_cast<size_t>(staged[j]);
-            if (cudaMemcpyAsync(dst + j * one.gu_bytes, src + e * one.gu_bytes, one.gu_bytes,
-                                cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-                cudaMemcpyAsync(dst + stg.gu_bytes + j * one.dn_bytes,
-                                src + all.gu_bytes + e * one.dn_bytes, one.dn_bytes,
-                                cudaMemcpyHostToDevice, cs) != cudaSuccess)
+            const char* se = src + static_cast<size_t>(staged[j]) * per_expert;
+            if (cudaMemcpyAsync(dst + j * one.gu_bytes, se, one.gu_bytes, cudaMemcpyHostToDevice,
+                                cs) != cudaSuccess ||
+                cudaMemcpyAsync(dst + stg.gu_bytes + j * one.dn_bytes, se + one.gu_bytes,
+                                one.dn_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
                 return MOE_ERR_CUDA;
         }
         if (a->copy_event &&
