@@ -19,7 +19,7 @@
  * it by slot and runs the resident and copied experts in its grouped GEMMs;
  * the host's rows join the combine.  bf16 only.  The conventions of moe.h
  * apply, with the exceptions stated at moe_split_forward (it synchronises its
- * stream once and reads and writes host memory).
+ * stream, once or twice, and reads and writes host memory).
  *
  * Process-wide state: the host functions share one thread pool (one thread
  * per hardware thread, created on first use, one pool per process: a child
@@ -164,9 +164,10 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
 
 /*
  * The split layer, for one batch x [T,H], logits [T,E]:
- *   1. GPU: route (a1) into ids, w; copy ids, w and x to the host; wait.
+ *   1. GPU: route (a1) into ids, w; copy ids and w to the host; wait.
  *   2. host: counts, then the plan (policy: moe_split_plan for DYNAMIC,
- *      moe_split_plan_balanced for BALANCED).
+ *      moe_split_plan_balanced for BALANCED); if the plan puts any expert on
+ *      the host, x is copied to the host (a second wait, for that copy).
  *   3. GPU: copy each STAGED expert's packed weights into a staging slot;
  *      map every assignment to a slot (0 = host, 1..S = the resident experts
  *      in ascending index, S+1.. = staged experts in ascending index) and
@@ -207,9 +208,10 @@ MOE_API moe_status moe_host_expert_ffn(const moe_host_ffn_args* args);
  * Calls that share staging slots or workspaces must be ordered: issue them
  * on one stream (each call's synchronisation then covers the previous one's
  * use of the slots).
- * Exceptions to moe.h's conventions: this call synchronises `stream` once
- * (after step 1: the plan needs the batch's routing) and computes on the
- * calling thread and the host pool; it returns once steps 3-5 are enqueued.
+ * Exceptions to moe.h's conventions: this call synchronises `stream` (after
+ * step 1: the plan needs the batch's routing; and for the copy of x when a
+ * host expert needs it) and computes on the calling thread and the host
+ * pool; it returns once steps 3-5 are enqueued.
  * Errors: as moe_forward; MOE_ERR_UNSUPPORTED for S + n_stage + 1 > 256.
  */
 typedef struct {

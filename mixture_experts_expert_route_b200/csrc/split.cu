@@ -277,8 +277,6 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
                 cudaSuccess ||
             cudaMemcpyAsync(hb.w, d.w, sizeof(float) * A, cudaMemcpyDeviceToHost, s) !=
                 cudaSuccess ||
-            cudaMemcpyAsync(hb.x, a->x, sizeof(uint16_t) * T * static_cast<size_t>(H),
-                            cudaMemcpyDeviceToHost, s) != cudaSuccess ||
             cudaStreamSynchronize(s) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
@@ -307,6 +305,27 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     }
     if (st != MOE_OK) return st;
     if (a->where) std::memcpy(a->where, where.data(), sizeof(int32_t) * E);
+
+    // the host experts' assignments, bucketed by expert in ascending flat
+    // index; x comes to the host only when some expert runs there (the stream
+    // is idle at this point, so the wait is for this copy alone)
+    std::vector<std::vector<long>> host_rows(E);
+    std::vector<int> pos(A, -1);
+    int n_cpu = 0;
+    for (long f = 0; f < A; ++f) {
+        const int e = hb.ids[f];
+        if (where[e] == MOE_SPLIT_CPU) {
+            pos[f] = n_cpu++;
+            host_rows[e].push_back(f);
+        }
+    }
+    if (n_cpu > 0) {
+        Range r("moe split: x to the host");
+        if (cudaMemcpyAsync(hb.x, a->x, sizeof(uint16_t) * T * static_cast<size_t>(H),
+                            cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
 
     // 3. slots, weight copies, slot permutation, the GPU experts
     Range gpu_part("moe split: weight copies, slot permutation, GPU experts");
@@ -375,18 +394,11 @@ moe_status moe_split_forward(const moe_split_args* a, void* ws, size_t ws_bytes,
     // 4. the host experts, while the GPU runs; their rows go to slot 0 in
     // ascending flat index, the order the stable permutation gives them
     Range host_part("moe split: host experts, combine");
-    std::vector<int> pos(A, -1);
-    int n_cpu = 0;
-    for (long f = 0; f < A; ++f)
-        if (where[hb.ids[f]] == MOE_SPLIT_CPU) pos[f] = n_cpu++;
     if (n_cpu > 0) {
         const size_t expert_bytes = moe_host_packed_size(H, I);
-        std::vector<long> rows;
         for (int e = 0; e < E; ++e) {
             if (where[e] != MOE_SPLIT_CPU) continue;
-            rows.clear();
-            for (long f = 0; f < A; ++f)
-                if (hb.ids[f] == e) rows.push_back(f);
+            const std::vector<long>& rows = host_rows[e];
             const int n = static_cast<int>(rows.size());
             for (int r = 0; r < n; ++r) {
                 std::memcpy(hb.xg + static_cast<size_t>(r) * H,
