@@ -52,7 +52,12 @@ def test_route_topk_bit_exact(moe, T, E, k):
                                            (64, 8, 2, 16, 0.0), (300, 32, 4, 64, 1.0),
                                            (1024, 128, 8, 16, 0.0), (4096, 128, 8, 128, 0.0),
                                            (8192, 256, 8, 16, 1.2), (5000, 7, 3, 32, 2.0),
-                                           (100, 256, 8, 16, 0.0)])
+                                           (100, 256, 8, 16, 0.0),
+                                           # chunk edges of the multi-CTA path (512 per chunk):
+                                           # one past the single-CTA limit, exact multiples,
+                                           # a last chunk of one assignment, E = 256 skewed
+                                           (2049, 8, 1, 16, 0.0), (1024, 64, 4, 16, 0.5),
+                                           (3073, 5, 1, 16, 0.0), (16384, 256, 2, 64, 1.5)])
 def test_align_permute_bit_exact(moe, T, E, k, bm, skew):
     ids = random_ids(T, E, k, seed=T + k, skew=skew)
     perm = moe.align_permute(ids.to(DEV), E, bm)

@@ -106,6 +106,35 @@ def test_many_experts_and_repeated_calls():
     run_case(300, 16, 4, 256, 384, resident, 3, 0, COSTS, seed=7, skew=0.5, calls=3)
 
 
+def test_block_m_and_one_host_thread():
+    moe = lib()
+    Wg, Wu, Wd, x, logits = make(90, 8, 2, 128, 256, seed=10)
+    layer = moe.SplitLayer(Wg, Wu, Wd, 2, [1, 0, 0, 1, 0, 0, 0, 0], n_stage=2, policy=0,
+                           costs=moe.split_costs(**COSTS), block_m=64, host_threads=1)
+    out = layer(x.cuda(), logits.cuda())
+    torch.cuda.synchronize()
+    assert layer.check() == 0
+    ids, w = oracle.route_topk(logits, 2)
+    assert list(layer.where) == expected_plan(ids, 8, [1, 0, 0, 1, 0, 0, 0, 0], 0, COSTS, 2, moe)
+    assert_close(out, oracle.moe_layer(x, ids, w, Wg, Wu, Wd), 0, "split block_m=64")
+
+
+def test_many_experts_top8():
+    # E = 256, k = 8: 1 + 40 + 16 slots, several host experts per batch
+    resident = [1 if e % 7 == 0 else 0 for e in range(256)]
+    run_case(128, 256, 8, 128, 128, resident, 16, 0, COSTS, seed=11, skew=0.5)
+
+
+def test_zero_tokens():
+    moe = lib()
+    Wg, Wu, Wd, x, logits = make(4, 4, 2, 64, 64, seed=12)
+    layer = moe.SplitLayer(Wg, Wu, Wd, 2, [1, 0, 0, 0], n_stage=1,
+                           costs=moe.split_costs(**COSTS))
+    out = layer(x[:0].cuda(), logits[:0].cuda())
+    torch.cuda.synchronize()
+    assert out.shape == (0, 64) and layer.check() == 0
+
+
 def test_calibrate():
     moe = lib()
     Wg, Wu, Wd, _, _ = make(1, 4, 2, 256, 512, seed=8)
