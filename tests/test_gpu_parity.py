@@ -57,7 +57,10 @@ def test_route_topk_bit_exact(moe, T, E, k):
                                            # one past the single-CTA limit, exact multiples,
                                            # a last chunk of one assignment, E = 256 skewed
                                            (2049, 8, 1, 16, 0.0), (1024, 64, 4, 16, 0.5),
-                                           (3073, 5, 1, 16, 0.0), (16384, 256, 2, 64, 1.5)])
+                                           (3073, 5, 1, 16, 0.0), (16384, 256, 2, 64, 1.5),
+                                           # small batches: E above 32, every expert, E = 1
+                                           (16, 8, 2, 16, 0.0), (3, 256, 8, 16, 0.0),
+                                           (4, 8, 8, 32, 0.0), (31, 1, 1, 16, 0.0)])
 def test_align_permute_bit_exact(moe, T, E, k, bm, skew):
     ids = random_ids(T, E, k, seed=T + k, skew=skew)
     perm = moe.align_permute(ids.to(DEV), E, bm)
@@ -144,6 +147,9 @@ LAYER_CASES = [
     ("tiny", 9, 1, 1, 256, 256),         # E = 1: dense SwiGLU
     ("tiny", 40, 2, 2, 256, 256),        # pair tiles, token cap 2*mean = 80 (not a multiple of 32)
     ("tiny", 56, 2, 2, 192, 128),        # pair tiles, 2*mean = 112
+    # small batches: 32 assignments, and E above 32 with k = 8
+    ("tiny", 16, 8, 2, 256, 256),
+    ("tiny", 3, 64, 8, 128, 128),
     # past the single-CTA permutation (T*k > 2048): route, count, scan+scatter
     ("tiny", 1100, 8, 2, 256, 256),      # 5 chunks, pair tiles (gather kernel between)
     ("tiny", 300, 128, 8, 128, 128),     # 5 chunks, one-CTA tiles: the GEMM follows scan+scatter
