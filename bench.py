@@ -127,7 +127,7 @@ def traffic_for(workload, T):
     """(bytes or None, note) for the roofline's `traffic` field."""
     rec = TRAFFIC.get((workload, T))
     if rec is None:
-        return None, NO_TRAFFIC.get(workload, "no ncu capture of this build")
+        return None, NO_TRAFFIC.get(workload, "no ncu capture of this GEMM code")
     if rec["gemm_src"] != gemm_source_hash():
         return None, f"stale: captured on GEMM sources {rec['gemm_src']} ({rec['capture']})"
     return rec["bytes"], f"ncu capture offline ({rec['capture']}), GEMM sources {rec['gemm_src']}"
