@@ -992,12 +992,19 @@ def run_native(args):
     head = headline_name(args)
     Ts = tuple(int(t) for t in args.Ts.split(",")) if args.Ts else None
     if head == "split":
+        # one GPU and its host: with several ranks the host cores would be
+        # shared between them, so only rank 0 measures
         clk.__exit__(None, None, None)
-        blk = run_split(args, dev, uuid)
         if rank == 0:
+            blk = run_split(args, dev, uuid)
             print(json.dumps({"metric": "CPU/GPU split layer tokens/s", **blk,
-                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                              "higher_is_better": True}), flush=True)
+                              "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                              "higher_is_better": True,
+                              "note": f"measured on rank 0 of {world}" if world > 1 else None}),
+                  flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
         return
 
     b = Bench(head, args, dev, dist, world, Ts)
