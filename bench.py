@@ -1003,8 +1003,7 @@ def run_native(args):
                               "note": f"measured on rank 0 of {world}" if world > 1 else None}),
                   flush=True)
         if dist:
-            dist.barrier()
-            dist.destroy_process_group()
+            dist.destroy_process_group()   # no barrier: rank 0's run outlasts the timeout
         return
 
     b = Bench(head, args, dev, dist, world, Ts)
