@@ -224,3 +224,35 @@ def test_host_kernel_in_a_forked_child(L):
             pytest.fail("the forked child did not finish")
         time.sleep(0.05)
     assert os.WIFEXITED(status) and os.WEXITSTATUS(status) == 0
+
+
+def test_calibrate_and_sizes_argument_errors(L):
+    import ctypes
+    lib = L.lib()
+    costs = L._lib.SplitCosts()
+    fake = ctypes.c_void_p(0x1000)
+    # bad sizes, missing buffers, a host workspace too small: nothing runs
+    assert lib.moe_split_calibrate(64, 100, 4, fake, fake, fake, fake, 1 << 20, 0, None,
+                                   ctypes.byref(costs)) == 1
+    assert lib.moe_split_calibrate(64, 64, 0, fake, fake, fake, fake, 1 << 20, 0, None,
+                                   ctypes.byref(costs)) == 1
+    assert lib.moe_split_calibrate(64, 64, 4, None, fake, fake, fake, 1 << 20, 0, None,
+                                   ctypes.byref(costs)) == 1
+    need = lib.moe_split_host_workspace_size(4, 1, 64, 64)
+    assert need > 0
+    assert lib.moe_split_calibrate(64, 64, 4, fake, fake, fake, fake, need - 1, 0, None,
+                                   ctypes.byref(costs)) == 3
+    # workspace sizes: resident count above E, staging slots past 256 slots, bad dims
+    assert lib.moe_split_workspace_size(8, 2, 8, 9, 1, 128, 128, 0) == 0
+    assert lib.moe_split_workspace_size(8, 2, 8, 8, 247, 128, 128, 0) > 0      # 1 + 8 + 247
+    assert lib.moe_split_workspace_size(8, 2, 8, 8, 248, 128, 128, 0) == 0
+    assert lib.moe_split_workspace_size(8, 2, 8, 4, 2, 100, 128, 0) == 0
+    assert lib.moe_split_host_workspace_size(8, 0, 128, 128) == 0
+    # plans and placement past 256 experts
+    big = np.zeros(257, np.int32)
+    assert lib.moe_split_plan(big.ctypes.data, big.ctypes.data, 257, ctypes.byref(costs), 1,
+                              big.ctypes.data) == 1
+    assert lib.moe_split_plan_balanced(big.ctypes.data, big.ctypes.data, 257,
+                                       ctypes.byref(costs), 1, big.ctypes.data) == 1
+    hits = np.zeros(257, np.int64)
+    assert lib.moe_split_place(hits.ctypes.data, 257, 1, big.ctypes.data) == 1
