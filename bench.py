@@ -1064,11 +1064,30 @@ def run_native(args):
         dist.destroy_process_group()
 
 
+def run_split_calls(args):
+    """Profiling mode of the split: N calls of the split layer at one T (the
+    dynamic plan with the latency model measured at set-up), for a profiler."""
+    import mixture_experts_expert_route_b200 as moe
+    T = int(args.Ts.split(",")[0]) if args.Ts else 64
+    dev = torch.device("cuda", 0)
+    sb = SplitBench(args, dev, Ts=(T,))
+    x, lg = sb.dev_in[T][0]
+    for _ in range(args.calls):
+        sb.layer(x, lg, out=sb.outs[T])
+    torch.cuda.synchronize()
+    if sb.layer.check() != 0:
+        raise RuntimeError("device status word reports a fault")
+    print(f"split T={T}: {args.calls} calls, plan {[int(v) for v in sb.layer.where]}", flush=True)
+
+
 def run_calls(args):
     """Profiling mode: N forward calls of one workload at one T (no timing, no
     JSON), for a profiler to capture; the weights are drawn on the GPU."""
     import mixture_experts_expert_route_b200 as moe
     name = headline_name(args)
+    if name == "split":
+        run_split_calls(args)
+        return
     wl = WORKLOADS[name]
     cfg = CONFIGS[wl["cfg"]]
     T = int(args.Ts.split(",")[0]) if args.Ts else max(cfg["T"])
